@@ -1,0 +1,378 @@
+/*
+ * fqa_oracle.c -- plain, slow CPU checker for the FP8 quantized attention path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may call, link or
+ * load this file: only the tests, the package's smoke check and the
+ * benchmark's CPU-baseline / reference arm use it.  It shares no code, header,
+ * table or constant with the CUDA library.
+ *
+ * What it computes (sources, by page title and section):
+ *  - Scaled dot-product attention with Q, K and V quantized to FP8, attention
+ *    kept in FP8 for numerical stability: "NVIDIA RTX AI optimiert FLUX.1 fuer
+ *    Bilddaten mit niedriger Genauigkeit" (the SDPA quantization paragraph and
+ *    the Table-1 paragraph) and "NVIDIA RTX AI, 저정밀 양자화로 FLUX.1 Kontext
+ *    최적화" (the SDPA paragraph).  SageAttention is named there as the lineage.
+ *  - The pages fix no scale granularity, smoothing, rounding or P rule.  This
+ *    file follows the readings stated beside each function: per-64-token-block
+ *    per-head absmax scales onto the E4M3 maximum 448, K smoothed by its
+ *    per-channel mean, KV tiles of Bc keys in ascending order with an exact
+ *    running maximum, P = E4M3(p * 448 * sv_J / sv_max), row sum of the
+ *    unquantized p, output scaled by sv_max / 448 / l.
+ *
+ * Precision: the quantizer runs in IEEE binary32 in a pinned operation order
+ * (compile with -ffp-contract=off, no fast-math) so that codes and scales are
+ * exact; attention runs in binary64 with roundings only at the pinned
+ * quantization points.  E4M3 follows the OCP 8-bit floating point
+ * specification (E4M3: bias 7, no infinities, NaN = S.1111.111, largest finite
+ * 448, subnormal step 2^-9); BF16 output rounding is round-to-nearest-even.
+ *
+ * Multithreaded with OpenMP over independent heads / query rows only; each
+ * result is computed by one thread in the order written here.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+#include <stdlib.h>
+
+#define ORC_E4M3_MAX 448.0
+
+/* ---------------------------------------------------------------- codecs */
+
+/* OCP E4M3: value of an 8-bit code. NaN codes (S.1111.111) return NaN. */
+double orc_e4m3_decode(uint8_t code)
+{
+    int sign = code >> 7;
+    int e = (code >> 3) & 0xF;
+    int m = code & 0x7;
+    double v;
+    if (e == 0xF && m == 0x7)
+        return NAN;
+    if (e == 0)
+        v = ldexp((double)m, -9);              /* subnormal: m/8 * 2^-6 */
+    else
+        v = ldexp(1.0 + m / 8.0, e - 7);
+    return sign ? -v : v;
+}
+
+/* OCP E4M3, round to nearest (ties to even), saturating to +-448.
+ * x must not be NaN.  The sign of zero is kept (-0 -> 0x80). */
+uint8_t orc_e4m3_encode(double x)
+{
+    uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    double a = fabs(x);
+    if (a >= ORC_E4M3_MAX)                       /* includes +inf */
+        return sign | 0x7E;
+    if (a < ldexp(1.0, -6)) {
+        /* subnormal range: multiples of 2^-9; q = 8 is the smallest normal,
+         * whose encoding (exponent field 1, mantissa 0) is also 8. */
+        double q = nearbyint(a * 512.0);
+        return sign | (uint8_t)q;
+    }
+    int e;
+    frexp(a, &e);                                /* a = f * 2^e, 0.5 <= f < 1 */
+    e -= 1;                                      /* a in [2^e, 2^(e+1)) */
+    double q = nearbyint(ldexp(a, 3 - e));       /* in [8, 16] */
+    if (q == 16.0) { q = 8.0; e += 1; }
+    if (e > 8 || (e == 8 && q > 14.0))           /* rounded above 448 */
+        return sign | 0x7E;
+    return sign | (uint8_t)(((e + 7) << 3) | ((int)q - 8));
+}
+
+/* BF16 bit pattern -> float (exact). */
+float orc_bf16_to_float(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+/* binary64 -> BF16, one round to nearest even (finite, normal-range inputs;
+ * subnormal results are rounded on the same 2^-133 grid). */
+uint16_t orc_bf16_round(double x)
+{
+    if (x == 0.0)
+        return signbit(x) ? 0x8000 : 0x0000;
+    int e;
+    double f = frexp(x, &e);                     /* 0.5 <= |f| < 1 */
+    if (e < -125) {                              /* below the normal range */
+        double q = nearbyint(ldexp(x, 133));
+        float r = (float)ldexp(q, -133);
+        uint32_t u; memcpy(&u, &r, 4);
+        return (uint16_t)(u >> 16);
+    }
+    double q = nearbyint(f * 256.0);             /* 8 significant bits */
+    float r = (float)ldexp(q, e - 8);            /* exact */
+    uint32_t u; memcpy(&u, &r, 4);
+    return (uint16_t)(u >> 16);
+}
+
+/* ------------------------------------------------------------- quantizer */
+
+#define IDX4(b, h, n, c, H, N, d) ((((size_t)(b) * (H) + (h)) * (N) + (n)) * (d) + (c))
+
+/* K per-channel mean, pinned order [reading: the pages give no summation
+ * order]: p_j[c] = ((0 + k[64j][c]) + k[64j+1][c]) + ... in binary32 over the
+ * 64 tokens of block j; T[c] = ((0 + p_0[c]) + p_1[c]) + ... over blocks;
+ * mu[c] = T[c] / (float)N, one binary32 division. */
+void orc_k_mean(const uint16_t *k, int B, int H, int N, int d, float *mu)
+{
+    int nblk = N / 64;
+    #pragma omp parallel for collapse(2) schedule(static)
+    for (int b = 0; b < B; b++)
+        for (int h = 0; h < H; h++)
+            for (int c = 0; c < d; c++) {
+                float T = 0.0f;
+                for (int j = 0; j < nblk; j++) {
+                    float p = 0.0f;
+                    for (int n = 64 * j; n < 64 * j + 64; n++)
+                        p = p + orc_bf16_to_float(k[IDX4(b, h, n, c, H, N, d)]);
+                    T = T + p;
+                }
+                mu[((size_t)b * H + h) * d + c] = T / (float)N;
+            }
+}
+
+/* One 64-token block of one head: absmax scale onto 448 and E4M3 codes.
+ * x[n*d + c] are the binary32 values to quantize.  Readings: s = amax/448 and
+ * inv = 448/amax as binary32 divisions; amax == 0 gives s = inv = 0; the
+ * code is E4M3_RNE_sat(fl32(x * inv)) -- the product is rounded to binary32
+ * first, then encoded. */
+static void quantize_block(const float *x, int d, uint8_t *codes, float *scale)
+{
+    float amax = 0.0f;
+    for (int i = 0; i < 64 * d; i++) {
+        float a = fabsf(x[i]);
+        if (a > amax) amax = a;
+    }
+    float s = 0.0f, inv = 0.0f;
+    if (amax > 0.0f) {
+        s = amax / 448.0f;
+        inv = 448.0f / amax;
+    }
+    for (int i = 0; i < 64 * d; i++) {
+        float y = x[i] * inv;
+        codes[i] = orc_e4m3_encode((double)y);
+    }
+    *scale = s;
+}
+
+/* The whole quantizer.  Inputs BF16 [B,H,N,d]; codes written in the same
+ * natural [B,H,N,d] layout (the CUDA library's own V layout is its business);
+ * sq, sk, sv: [B,H,N/64]; sv_max: [B,H]; k_mean: [B,H,d].
+ * K is smoothed as fl32(k - mu[c]) before its block scales are taken. */
+void orc_quantize(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                  int B, int H, int N, int d,
+                  uint8_t *q8, uint8_t *k8, uint8_t *v8,
+                  float *sq, float *sk, float *sv, float *sv_max, float *k_mean)
+{
+    int nblk = N / 64;
+    orc_k_mean(k, B, H, N, d, k_mean);
+    #pragma omp parallel for collapse(2) schedule(dynamic)
+    for (int b = 0; b < B; b++)
+        for (int h = 0; h < H; h++) {
+            float *x = (float *)malloc(sizeof(float) * 64 * d);
+            const float *mu = k_mean + ((size_t)b * H + h) * d;
+            float vmax = 0.0f;
+            for (int j = 0; j < nblk; j++) {
+                size_t base = IDX4(b, h, 64 * j, 0, H, N, d);
+                size_t sidx = ((size_t)b * H + h) * nblk + j;
+                for (int i = 0; i < 64 * d; i++)
+                    x[i] = orc_bf16_to_float(q[base + i]);
+                quantize_block(x, d, q8 + base, &sq[sidx]);
+                for (int i = 0; i < 64 * d; i++)
+                    x[i] = orc_bf16_to_float(k[base + i]) - mu[i % d];
+                quantize_block(x, d, k8 + base, &sk[sidx]);
+                for (int i = 0; i < 64 * d; i++)
+                    x[i] = orc_bf16_to_float(v[base + i]);
+                quantize_block(x, d, v8 + base, &sv[sidx]);
+                if (sv[sidx] > vmax) vmax = sv[sidx];
+            }
+            sv_max[(size_t)b * H + h] = vmax;
+            free(x);
+        }
+}
+
+/* ------------------------------------------------------------- attention */
+
+/* Tiled attention core in binary64 for one head, on already dequantized
+ * operands: qc [N,d], kc [N,d], vc [N,d] are the code VALUES (not yet
+ * multiplied by their block scales), sq/sk/sv the per-64-token scales.
+ *
+ * For query row i (block I = i/64), KV tiles t of bc keys in ascending order:
+ *   x_ij   = (sum_c qc_ic kc_jc) * sq_I * sk_J * scale * log2(e)
+ *   m_t    = max(m_{t-1}, max_{j in t} x_ij),  m_{-1} = -inf  (exact, no
+ *            threshold / lazy rescale)
+ *   p_ij   = 2^(x_ij - m_t)
+ *   P_ij   = E4M3(p_ij * 448 * sv_J / sv_max)    [quantize_p != 0]
+ *          = p_ij * 448 * sv_J / sv_max          [quantize_p == 0]
+ *   l      = l * 2^(m_{t-1} - m_t) + sum_j p_ij   (unquantized p)
+ *   acc_c  = acc_c * 2^(m_{t-1} - m_t) + sum_j P_ij vc_jc
+ *   O_ic   = acc_c * (sv_max / 448) / l
+ * sv_max == 0 (V entirely zero) gives O = 0.
+ * rows: the query rows of this head to evaluate; out: [n_rows, d]. */
+static void attention_core_head(const double *qc, const double *kc, const double *vc,
+                                const float *sq, const float *sk, const float *sv, float sv_max,
+                                int N, int d, double scale, int bc, int quantize_p,
+                                const int *rows, int n_rows, double *out)
+{
+    const double LOG2E = 1.4426950408889634073599246810019;  /* log2(e) */
+    #pragma omp parallel for schedule(dynamic, 4)
+    for (int r = 0; r < n_rows; r++) {
+        int i = rows[r];
+        double *o = out + (size_t)r * d;
+        double *x = (double *)malloc(sizeof(double) * bc);
+        double *acc = (double *)calloc(d, sizeof(double));
+        double m = -INFINITY, l = 0.0;
+        if (sv_max == 0.0f) {
+            for (int c = 0; c < d; c++) o[c] = 0.0;
+            free(x); free(acc);
+            continue;
+        }
+        for (int t0 = 0; t0 < N; t0 += bc) {
+            int t1 = t0 + bc < N ? t0 + bc : N;
+            double tmax = -INFINITY;
+            for (int j = t0; j < t1; j++) {
+                double s = 0.0;
+                for (int c = 0; c < d; c++)
+                    s += qc[(size_t)i * d + c] * kc[(size_t)j * d + c];
+                x[j - t0] = s * (double)sq[i / 64] * (double)sk[j / 64] * scale * LOG2E;
+                if (x[j - t0] > tmax) tmax = x[j - t0];
+            }
+            double m_new = tmax > m ? tmax : m;
+            double alpha = exp2(m - m_new);      /* 0 on the first tile */
+            l *= alpha;
+            for (int c = 0; c < d; c++) acc[c] *= alpha;
+            for (int j = t0; j < t1; j++) {
+                double p = exp2(x[j - t0] - m_new);
+                double rv = (double)sv[j / 64] / (double)sv_max;
+                double P = p * 448.0 * rv;
+                if (quantize_p)
+                    P = orc_e4m3_decode(orc_e4m3_encode(P));
+                l += p;
+                for (int c = 0; c < d; c++)
+                    acc[c] += P * vc[(size_t)j * d + c];
+            }
+            m = m_new;
+        }
+        for (int c = 0; c < d; c++)
+            o[c] = acc[c] * ((double)sv_max / 448.0) / l;
+        free(x);
+        free(acc);
+    }
+}
+
+/* Exported core for the pins: operands given as binary64 values. */
+void orc_attention_core(const double *qc, const double *kc, const double *vc,
+                        const float *sq, const float *sk, const float *sv, float sv_max,
+                        int N, int d, double scale, int bc, int quantize_p,
+                        const int *rows, int n_rows, double *out)
+{
+    attention_core_head(qc, kc, vc, sq, sk, sv, sv_max, N, d, scale, bc, quantize_p,
+                        rows, n_rows, out);
+}
+
+/* FP8 attention on quantizer outputs (codes in natural [B,H,N,d] layout).
+ * heads: n_heads pairs (b, h); rows: n_rows query rows evaluated in every
+ * listed head; out: [n_heads, n_rows, d] binary64. */
+void orc_attention_fp8(const uint8_t *q8, const uint8_t *k8, const uint8_t *v8,
+                       const float *sq, const float *sk, const float *sv, const float *sv_max,
+                       int B, int H, int N, int d, float softmax_scale, int bc,
+                       const int *heads, int n_heads, const int *rows, int n_rows,
+                       double *out)
+{
+    int nblk = N / 64;
+    (void)B;
+    double *qc = (double *)malloc(sizeof(double) * N * d);
+    double *kc = (double *)malloc(sizeof(double) * N * d);
+    double *vc = (double *)malloc(sizeof(double) * N * d);
+    double dec[256];
+    for (int i = 0; i < 256; i++) dec[i] = orc_e4m3_decode((uint8_t)i);
+    for (int hh = 0; hh < n_heads; hh++) {
+        int b = heads[2 * hh], h = heads[2 * hh + 1];
+        size_t base = IDX4(b, h, 0, 0, H, N, d);
+        for (size_t i = 0; i < (size_t)N * d; i++) {
+            qc[i] = dec[q8[base + i]];
+            kc[i] = dec[k8[base + i]];
+            vc[i] = dec[v8[base + i]];
+        }
+        size_t sidx = ((size_t)b * H + h) * nblk;
+        attention_core_head(qc, kc, vc, sq + sidx, sk + sidx, sv + sidx,
+                            sv_max[(size_t)b * H + h], N, d, (double)softmax_scale, bc, 1,
+                            rows, n_rows, out + (size_t)hh * n_rows * d);
+    }
+    free(qc); free(kc); free(vc);
+}
+
+/* Exact attention, binary64, no quantization: softmax(Q K^T * scale) V on the
+ * BF16 inputs with a two-pass row maximum.  Same heads/rows/out convention. */
+void orc_attention_exact(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                         int B, int H, int N, int d, double scale,
+                         const int *heads, int n_heads, const int *rows, int n_rows,
+                         double *out)
+{
+    (void)B;
+    double *kd = (double *)malloc(sizeof(double) * N * d);
+    double *vd = (double *)malloc(sizeof(double) * N * d);
+    for (int hh = 0; hh < n_heads; hh++) {
+        int b = heads[2 * hh], h = heads[2 * hh + 1];
+        size_t base = IDX4(b, h, 0, 0, H, N, d);
+        for (size_t i = 0; i < (size_t)N * d; i++) {
+            kd[i] = orc_bf16_to_float(k[base + i]);
+            vd[i] = orc_bf16_to_float(v[base + i]);
+        }
+        #pragma omp parallel for schedule(dynamic, 4)
+        for (int r = 0; r < n_rows; r++) {
+            int i = rows[r];
+            double *o = out + ((size_t)hh * n_rows + r) * d;
+            double *s = (double *)malloc(sizeof(double) * N);
+            double qi[512];
+            for (int c = 0; c < d && c < 512; c++)
+                qi[c] = orc_bf16_to_float(q[base + (size_t)i * d + c]);
+            double mx = -INFINITY;
+            for (int j = 0; j < N; j++) {
+                double acc = 0.0;
+                for (int c = 0; c < d; c++) acc += qi[c] * kd[(size_t)j * d + c];
+                s[j] = acc * scale;
+                if (s[j] > mx) mx = s[j];
+            }
+            double l = 0.0;
+            for (int c = 0; c < d; c++) o[c] = 0.0;
+            for (int j = 0; j < N; j++) {
+                double p = exp(s[j] - mx);
+                l += p;
+                for (int c = 0; c < d; c++) o[c] += p * vd[(size_t)j * d + c];
+            }
+            for (int c = 0; c < d; c++) o[c] /= l;
+            free(s);
+        }
+    }
+    free(kd); free(vd);
+}
+
+/* Vectorised encoder over binary32 inputs, for the exhaustive codec check
+ * against the GPU's conversion instruction. */
+void orc_e4m3_encode_f32_array(const float *x, size_t n, uint8_t *out)
+{
+    #pragma omp parallel for schedule(static)
+    for (size_t i = 0; i < n; i++)
+        out[i] = isnan(x[i]) ? 0x7F : orc_e4m3_encode((double)x[i]);
+}
+
+/* Vectorised BF16 rounding of binary64 values. */
+void orc_bf16_round_array(const double *x, size_t n, uint16_t *out)
+{
+    #pragma omp parallel for schedule(static)
+    for (size_t i = 0; i < n; i++)
+        out[i] = orc_bf16_round(x[i]);
+}
+
+int orc_num_threads(void)
+{
+#ifdef _OPENMP
+    extern int omp_get_max_threads(void);
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
