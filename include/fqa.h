@@ -1,0 +1,179 @@
+/*
+ * fqa.h -- C ABI of the FP8 quantized attention library for B200 (sm_100a).
+ *
+ * The library computes the hot path of FLUX-style diffusion-transformer
+ * inference: non-causal scaled dot-product attention over the joint
+ * text + image (+ context-image) token sequence, with Q, K and V quantized to
+ * FP8 E4M3 and the attention itself run in FP8, plus an unquantized BF16
+ * comparison path.
+ *
+ * Sources (web pages, by title and section):
+ *  [RTX-DE] "NVIDIA RTX AI optimiert FLUX.1 fuer Bilddaten mit niedriger
+ *           Genauigkeit": the SDPA quantization paragraph (FP8 and FP4 schemes
+ *           differ only in the precision of the Q, K, V projections;
+ *           SageAttention named as the lineage) and the Table-1 paragraph
+ *           (attention kept in FP8 for numerical stability; FP8 about 2x BF16).
+ *  [RTX-KR] "NVIDIA RTX AI, 저정밀 양자화로 FLUX.1 Kontext 최적화": SDPA is about
+ *           75% of the transformer's compute cost; quantizing it is the core
+ *           of the work; Kontext concatenates context-image tokens (about 2x
+ *           the sequence).
+ *  [KLEIN]  "FLUX 3 Image Klein Base: 생성 3.46배, 8장 확장 병목", section
+ *           "왜 이런 차이가 나나": VANILLA BF16 attention is about 60% of DiT
+ *           kernel time on one B200; cuDNN FP8 and VC-Attention FP8 are the
+ *           FP8 backends measured there.
+ * The pages give no scale granularity, smoothing, rounding, P rule or API.
+ * The readings used (stated again at each call): one FP32 absmax scale per
+ * (batch, head, 64-token block) mapping onto the E4M3 maximum 448, K smoothed
+ * by its per-channel mean, KV tiles of 128 keys with an exact running maximum,
+ * P = E4M3(p * 448 * sv_J / sv_max), row sum of unquantized p.
+ *
+ * Conventions for every call:
+ *  - Pointers named as tensors are DEVICE pointers owned by the caller; the
+ *    library allocates no device memory, frees nothing and keeps no per-call
+ *    state (a per-device cache of a status-word address and the driver's
+ *    tensor-map encoder is built on first use, thread-safely).
+ *  - All work is enqueued asynchronously on `cuda_stream` (a cudaStream_t;
+ *    NULL = the legacy default stream).  No call synchronizes, except
+ *    fqa_debug_status().
+ *  - Layouts are row-major and contiguous: [B, H, N, d] with d innermost.
+ *  - v1 limits: d == 128; N a multiple of 128 (quantizer: of 64);
+ *    1 <= N <= 65536; B, H >= 1, B*H <= 65535, B*H*N < 2^31; device pointers
+ *    16-byte aligned (scale arrays 4-byte aligned); a finite softmax_scale > 0;
+ *    outputs must not overlap inputs.
+ *  - Errors: arguments are checked on the host before anything is launched;
+ *    an argument error returns a status and launches nothing.  A launch
+ *    failure returns FQA_ERR_CUDA.  Non-finite input values are outside the
+ *    contract (no error is reported; results are unspecified).
+ *  - Device-side waits are bounded (about 1.5 s); a wait that gives up sets a
+ *    bit in a device status word, abandons the tile and returns; read it with
+ *    fqa_debug_status().  No kernel traps.
+ */
+#ifndef FQA_H
+#define FQA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FQA_API __attribute__((visibility("default")))
+#else
+#define FQA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FQA_OK = 0,
+  FQA_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, bad dtype, small workspace */
+  FQA_ERR_UNSUPPORTED = 2,  /* d != 128, N not a multiple of 128 (64), sizes beyond the limits */
+  FQA_ERR_MISALIGNED = 3,   /* a pointer not aligned as required */
+  FQA_ERR_CUDA = 4,         /* a CUDA runtime / driver call or launch failed */
+  FQA_ERR_TIMEOUT = 5       /* a bounded device wait gave up (from fqa_debug_status) */
+} fqa_status;
+
+typedef enum {
+  FQA_OUT_BF16 = 0,         /* production output, round to nearest even */
+  FQA_OUT_F32 = 1           /* verification output: the FP32 values before BF16 rounding */
+} fqa_out_dtype;
+
+/* Library version, (major << 16) | minor. */
+FQA_API int fqa_version(void);
+
+/* Human-readable name of a status code (static storage). */
+FQA_API const char* fqa_status_string(fqa_status status);
+
+/*
+ * Bytes of device workspace fqa_quantize() needs: B*H*(N/64)*d*4 (the
+ * per-64-token-block partial sums of the K mean).  Returns 0 for invalid
+ * sizes.
+ */
+FQA_API size_t fqa_quantize_workspace_bytes(int B, int H, int N, int d);
+
+/*
+ * fqa_quantize -- BF16 Q, K, V -> E4M3 codes and FP32 block scales.
+ * [RTX-DE] SDPA quantization paragraph: Q, K and V are the quantized inputs.
+ *
+ * For each (b, h):
+ *   k_mean[c] = (sum over 64-token blocks j, ascending, of the sequential
+ *               binary32 sum of K over the block's 64 tokens) / N
+ *               (pinned order, one round-to-nearest division);
+ *   for each 64-token block and tensor X in {Q, K - k_mean, V} (the K
+ *   difference is one binary32 subtraction per element):
+ *     amax = max |X| over the 64 x 128 block;
+ *     scale = amax / 448, inv = 448 / amax (binary32 divisions; both 0 if amax = 0);
+ *     code  = E4M3 round-to-nearest-even, saturating, of fl32(X * inv);
+ *   sv_max = max over blocks of the V scales.
+ * The results are bit-exact functions of the inputs (no atomics that change
+ * values, no order dependence).
+ *
+ * q, k, v      in : BF16 [B,H,N,d]
+ * q8, k8, v8   out: E4M3 codes, uint8 [B,H,N,d] (same layout as the inputs)
+ * sq, sk, sv   out: FP32 [B,H,N/64] block scales
+ * sv_max       out: FP32 [B,H]
+ * k_mean       out: FP32 [B,H,d]
+ * workspace    scratch of at least fqa_quantize_workspace_bytes(B,H,N,d)
+ *              bytes, 16-byte aligned; contents on entry are ignored.
+ * Launches three kernels on cuda_stream.
+ */
+FQA_API fqa_status fqa_quantize(const void* q, const void* k, const void* v, int B, int H, int N, int d,
+                        void* q8, void* k8, void* v8, float* sq, float* sk, float* sv,
+                        float* sv_max, float* k_mean, void* workspace, size_t workspace_bytes,
+                        void* cuda_stream);
+
+/*
+ * fqa_attention_fp8 -- fused FP8 attention on fqa_quantize() outputs.
+ * [RTX-DE] Table-1 paragraph (attention in FP8); [RTX-KR] SDPA paragraph.
+ *
+ * For query row i (64-token block I) over KV tiles of 128 keys, ascending:
+ *   x_j  = (q8_i . k8_j) * sq_I * sk_J * softmax_scale * log2(e)   (J = j/64)
+ *   m    = running max of x, updated exactly once per tile
+ *   p_j  = 2^(x_j - m),  l = l * 2^(m_old - m_new) + sum p_j
+ *   P_j  = E4M3(p_j * 448 * sv_J / sv_max)
+ *   O    = O * 2^(m_old - m_new) + sum_j P_j * v8_j        (FP32 accumulate)
+ *   out_i = O * (sv_max / 448) / l
+ * Scores use the smoothed K codes; smoothing leaves softmax unchanged because
+ * q . k_mean is constant along a row.  sv_max == 0 gives out = 0.
+ *
+ * out: [B,H,N,d] BF16 (FQA_OUT_BF16) or FP32 (FQA_OUT_F32).
+ * softmax_scale: typically fl32(1/sqrt(d)).
+ */
+FQA_API fqa_status fqa_attention_fp8(const void* q8, const void* k8, const void* v8, const float* sq,
+                             const float* sk, const float* sv, const float* sv_max, int B, int H,
+                             int N, int d, float softmax_scale, void* out,
+                             fqa_out_dtype out_dtype, void* cuda_stream);
+
+/*
+ * fqa_attention_bf16 -- the unquantized comparison path ([KLEIN], VANILLA
+ * BF16 attention): softmax(Q K^T * softmax_scale) V with BF16 operands, FP32
+ * accumulation and online softmax over 128-key tiles, P rounded to BF16 for
+ * the P.V product, out = O / l.
+ *
+ * q, k, v: BF16 [B,H,N,d]; out: [B,H,N,d] BF16 or FP32.
+ */
+FQA_API fqa_status fqa_attention_bf16(const void* q, const void* k, const void* v, int B, int H, int N,
+                              int d, float softmax_scale, void* out, fqa_out_dtype out_dtype,
+                              void* cuda_stream);
+
+/*
+ * fqa_e4m3_encode -- the library's binary32 -> E4M3 conversion (round to
+ * nearest even, saturating to +-448, NaN -> 0x7F), exposed so that callers
+ * can check the codec exhaustively.  x: FP32 [n], out: uint8 [n] (device).
+ */
+FQA_API fqa_status fqa_e4m3_encode(const float* x, uint8_t* out, size_t n, void* cuda_stream);
+
+/*
+ * fqa_debug_status -- synchronizes cuda_stream, reads and clears the
+ * device status word of the current device.  Returns FQA_ERR_TIMEOUT if a
+ * bounded device wait gave up since the last call, FQA_ERR_CUDA if the
+ * synchronization failed, FQA_OK otherwise.  *flags_out (if not NULL)
+ * receives the raw bits.
+ */
+FQA_API fqa_status fqa_debug_status(void* cuda_stream, uint32_t* flags_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FQA_H */

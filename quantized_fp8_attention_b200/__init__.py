@@ -1,0 +1,210 @@
+"""Python binding of libfqa.so, the B200 FP8 quantized attention library.
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels.  PyTorch provides device memory and the current stream.  The C ABI
+is declared (and documented) in include/fqa.h; the functions below carry the
+same names and pass ``tensor.data_ptr()`` and the stream handle through.
+
+The library must have been built (``python -m quantized_fp8_attention_b200.build``
+or ``__graft_entry__.build()``); every call raises ImportError without it.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import NamedTuple, Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libfqa.so")
+
+FQA_OK, FQA_ERR_INVALID_ARG, FQA_ERR_UNSUPPORTED, FQA_ERR_MISALIGNED, FQA_ERR_CUDA, FQA_ERR_TIMEOUT = range(6)
+FQA_OUT_BF16, FQA_OUT_F32 = 0, 1
+HEAD_DIM = 128
+
+_lib = None
+
+
+def _load():
+    """Load libfqa.so and declare the C signatures.  Raises if it is not built:
+    there is no fallback implementation."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"libfqa.so is not built ({LIB_PATH}); run `python -m quantized_fp8_attention_b200.build`. "
+            "There is no fallback implementation.")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I = ctypes.c_void_p, ctypes.c_int
+    L.fqa_version.restype = I
+    L.fqa_status_string.restype = ctypes.c_char_p
+    L.fqa_status_string.argtypes = [I]
+    L.fqa_quantize_workspace_bytes.restype = ctypes.c_size_t
+    L.fqa_quantize_workspace_bytes.argtypes = [I, I, I, I]
+    L.fqa_quantize.restype = I
+    L.fqa_quantize.argtypes = [P, P, P, I, I, I, I, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+    L.fqa_attention_fp8.restype = I
+    L.fqa_attention_fp8.argtypes = [P, P, P, P, P, P, P, I, I, I, I, ctypes.c_float, P, I, P]
+    L.fqa_attention_bf16.restype = I
+    L.fqa_attention_bf16.argtypes = [P, P, P, I, I, I, I, ctypes.c_float, P, I, P]
+    L.fqa_e4m3_encode.restype = I
+    L.fqa_e4m3_encode.argtypes = [P, P, ctypes.c_size_t, P]
+    L.fqa_debug_status.restype = I
+    L.fqa_debug_status.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
+    _lib = L
+    return L
+
+
+class FqaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+def lib():
+    """The loaded ctypes library (for tests that call the ABI directly)."""
+    return _load()
+
+
+def status_string(status: int) -> str:
+    return _load().fqa_status_string(int(status)).decode()
+
+
+def version() -> int:
+    return _load().fqa_version()
+
+
+def _check(status: int, where: str):
+    if status != FQA_OK:
+        raise FqaError(status, where)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+# ------------------------------------------------------------- raw ABI
+
+def fqa_quantize_workspace_bytes(B: int, H: int, N: int, d: int = HEAD_DIM) -> int:
+    return int(_load().fqa_quantize_workspace_bytes(B, H, N, d))
+
+
+def fqa_quantize(q, k, v, q8, k8, v8, sq, sk, sv, sv_max, k_mean, workspace, stream=None) -> int:
+    """The C call with tensors; returns the fqa_status code."""
+    B, H, N, d = q.shape
+    return _load().fqa_quantize(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, _ptr(q8), _ptr(k8), _ptr(v8),
+                             _ptr(sq), _ptr(sk), _ptr(sv), _ptr(sv_max), _ptr(k_mean),
+                             _ptr(workspace), workspace.numel() * workspace.element_size(),
+                             _stream(stream))
+
+
+def fqa_attention_fp8(q8, k8, v8, sq, sk, sv, sv_max, softmax_scale, out, out_dtype, stream=None) -> int:
+    B, H, N, d = q8.shape
+    return _load().fqa_attention_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(sq), _ptr(sk), _ptr(sv),
+                                  _ptr(sv_max), B, H, N, d, float(softmax_scale), _ptr(out),
+                                  int(out_dtype), _stream(stream))
+
+
+def fqa_attention_bf16(q, k, v, softmax_scale, out, out_dtype, stream=None) -> int:
+    B, H, N, d = q.shape
+    return _load().fqa_attention_bf16(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, float(softmax_scale),
+                                   _ptr(out), int(out_dtype), _stream(stream))
+
+
+def fqa_e4m3_encode(x, out, stream=None) -> int:
+    return _load().fqa_e4m3_encode(_ptr(x), _ptr(out), x.numel(), _stream(stream))
+
+
+def fqa_debug_status(stream=None):
+    """(status, raw flag bits) of the current device's status word; clears it."""
+    flags = ctypes.c_uint32(0)
+    st = _load().fqa_debug_status(_stream(stream), ctypes.byref(flags))
+    return st, flags.value
+
+
+# ----------------------------------------------------- tensor-level API
+
+class Quantized(NamedTuple):
+    q8: torch.Tensor       # uint8 E4M3 codes [B,H,N,128]
+    k8: torch.Tensor
+    v8: torch.Tensor
+    sq: torch.Tensor       # float32 [B,H,N/64]
+    sk: torch.Tensor
+    sv: torch.Tensor
+    sv_max: torch.Tensor   # float32 [B,H]
+    k_mean: torch.Tensor   # float32 [B,H,128]
+
+
+def alloc_quantized(B: int, H: int, N: int, device) -> Quantized:
+    u8 = dict(dtype=torch.uint8, device=device)
+    f32 = dict(dtype=torch.float32, device=device)
+    return Quantized(torch.empty(B, H, N, HEAD_DIM, **u8), torch.empty(B, H, N, HEAD_DIM, **u8),
+                     torch.empty(B, H, N, HEAD_DIM, **u8), torch.empty(B, H, N // 64, **f32),
+                     torch.empty(B, H, N // 64, **f32), torch.empty(B, H, N // 64, **f32),
+                     torch.empty(B, H, **f32), torch.empty(B, H, HEAD_DIM, **f32))
+
+
+def alloc_workspace(B: int, H: int, N: int, device) -> torch.Tensor:
+    nbytes = fqa_quantize_workspace_bytes(B, H, N)
+    return torch.empty(max(nbytes, 16) // 4, dtype=torch.float32, device=device)
+
+
+def quantize(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: Optional[Quantized] = None,
+             workspace: Optional[torch.Tensor] = None, stream=None) -> Quantized:
+    """BF16 [B,H,N,128] Q, K, V (CUDA, contiguous) -> Quantized."""
+    B, H, N, _ = q.shape
+    if out is None:
+        out = alloc_quantized(B, H, N, q.device)
+    if workspace is None:
+        workspace = alloc_workspace(B, H, N, q.device)
+    _check(fqa_quantize(q, k, v, *out, workspace, stream=stream), "fqa_quantize")
+    return out
+
+
+def attention_fp8(qz: Quantized, softmax_scale: float, out_dtype: int = FQA_OUT_BF16,
+                  out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    B, H, N, d = qz.q8.shape
+    if out is None:
+        dt = torch.float32 if out_dtype == FQA_OUT_F32 else torch.bfloat16
+        out = torch.empty(B, H, N, d, dtype=dt, device=qz.q8.device)
+    _check(fqa_attention_fp8(qz.q8, qz.k8, qz.v8, qz.sq, qz.sk, qz.sv, qz.sv_max, softmax_scale,
+                             out, out_dtype, stream=stream), "fqa_attention_fp8")
+    return out
+
+
+def attention_bf16(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, softmax_scale: float,
+                   out_dtype: int = FQA_OUT_BF16, out: Optional[torch.Tensor] = None,
+                   stream=None) -> torch.Tensor:
+    B, H, N, d = q.shape
+    if out is None:
+        dt = torch.float32 if out_dtype == FQA_OUT_F32 else torch.bfloat16
+        out = torch.empty(B, H, N, d, dtype=dt, device=q.device)
+    _check(fqa_attention_bf16(q, k, v, softmax_scale, out, out_dtype, stream=stream),
+           "fqa_attention_bf16")
+    return out
+
+
+def fp8_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, softmax_scale: float,
+                  out_dtype: int = FQA_OUT_BF16, stream=None) -> torch.Tensor:
+    """The whole FP8 path: quantize, then fused FP8 attention."""
+    return attention_fp8(quantize(q, k, v, stream=stream), softmax_scale, out_dtype, stream=stream)
+
+
+def e4m3_encode(x: torch.Tensor, stream=None) -> torch.Tensor:
+    out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    _check(fqa_e4m3_encode(x, out, stream=stream), "fqa_e4m3_encode")
+    return out
+
+
+def softmax_scale(d: int = HEAD_DIM) -> float:
+    """fl32(1/sqrt(d))."""
+    return float(torch.tensor(1.0, dtype=torch.float32) / torch.sqrt(torch.tensor(float(d), dtype=torch.float32)))

@@ -1,0 +1,239 @@
+// fqa.cu -- the library's C ABI (include/fqa.h): host-side argument checks,
+// TMA tensor-map encoding and kernel launches.  One translation unit holds
+// every kernel, so the device status word needs no relocatable device code.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/fqa.h"
+#include "attention.cuh"
+#include "device.cuh"
+#include "quantize.cuh"
+
+namespace fqa {
+
+__device__ uint32_t g_status_word;
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceCache {
+  std::once_flag once;
+  uint32_t* status = nullptr;
+  cudaError_t err = cudaSuccess;
+};
+DeviceCache g_dev[kMaxDevices];
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+std::once_flag g_encode_once;
+EncodeTiledFn g_encode = nullptr;
+
+static uint32_t* status_ptr(fqa_status* st) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    *st = FQA_ERR_CUDA;
+    return nullptr;
+  }
+  DeviceCache& c = g_dev[dev];
+  std::call_once(c.once, [&c]() {
+    void* p = nullptr;
+    c.err = cudaGetSymbolAddress(&p, g_status_word);
+    if (c.err == cudaSuccess) c.status = static_cast<uint32_t*>(p);
+  });
+  if (c.err != cudaSuccess || c.status == nullptr) {
+    *st = FQA_ERR_CUDA;
+    return nullptr;
+  }
+  return c.status;
+}
+
+static EncodeTiledFn encoder() {
+  std::call_once(g_encode_once, []() {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  });
+  return g_encode;
+}
+
+// 2-D view [rows, 128] of a [B,H,N,128] tensor; box = 128 rows x (128 B of
+// columns), 128-byte swizzle.
+static bool make_tmap(CUtensorMap* m, const void* base, bool fp8, uint64_t rows) {
+  EncodeTiledFn enc = encoder();
+  if (!enc) return false;
+  const uint32_t elt = fp8 ? 1 : 2;
+  cuuint64_t dims[2] = {128, rows};
+  cuuint64_t strides[1] = {128ull * elt};
+  cuuint32_t box[2] = {128u / elt, 128u};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                   const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+static bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Shape checks shared by every call. n_mult: required multiple of N.
+static fqa_status check_shape(int B, int H, int N, int d, int n_mult) {
+  if (B < 1 || H < 1 || N < 1 || d < 1) return FQA_ERR_INVALID_ARG;
+  if (d != 128) return FQA_ERR_UNSUPPORTED;
+  if (N % n_mult != 0 || N > 65536) return FQA_ERR_UNSUPPORTED;
+  if ((int64_t)B * H > 65535) return FQA_ERR_UNSUPPORTED;
+  if ((int64_t)B * H * N >= (int64_t(1) << 31)) return FQA_ERR_UNSUPPORTED;
+  return FQA_OK;
+}
+
+static fqa_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? FQA_OK : FQA_ERR_CUDA;
+}
+
+template <bool kFP8>
+static fqa_status launch_attention(const void* q, const void* k, const void* v, const AttnParams& prm,
+                                   cudaStream_t stream) {
+  using T = AttnTraits<kFP8>;
+  const uint64_t rows = (uint64_t)prm.B * prm.H * prm.N;
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap(&tq, q, kFP8, rows) || !make_tmap(&tk, k, kFP8, rows) ||
+      !make_tmap(&tv, v, kFP8, rows))
+    return FQA_ERR_CUDA;
+  auto kern = attn_fwd_kernel<kFP8>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, T::kSmemBytes) !=
+      cudaSuccess)
+    return FQA_ERR_CUDA;
+  dim3 grid(prm.N / kBlockM, prm.H, prm.B);
+  kern<<<grid, kAttnThreads, T::kSmemBytes, stream>>>(tq, tk, tv, prm);
+  return launch_status();
+}
+
+}  // namespace fqa
+
+using namespace fqa;
+
+extern "C" {
+
+int fqa_version(void) { return (1 << 16) | 0; }
+
+const char* fqa_status_string(fqa_status s) {
+  switch (s) {
+    case FQA_OK: return "FQA_OK";
+    case FQA_ERR_INVALID_ARG: return "FQA_ERR_INVALID_ARG";
+    case FQA_ERR_UNSUPPORTED: return "FQA_ERR_UNSUPPORTED";
+    case FQA_ERR_MISALIGNED: return "FQA_ERR_MISALIGNED";
+    case FQA_ERR_CUDA: return "FQA_ERR_CUDA";
+    case FQA_ERR_TIMEOUT: return "FQA_ERR_TIMEOUT";
+  }
+  return "FQA_UNKNOWN_STATUS";
+}
+
+size_t fqa_quantize_workspace_bytes(int B, int H, int N, int d) {
+  if (check_shape(B, H, N, d, kQBlock) != FQA_OK) return 0;
+  return (size_t)B * H * (N / kQBlock) * d * sizeof(float);
+}
+
+fqa_status fqa_quantize(const void* q, const void* k, const void* v, int B, int H, int N, int d,
+                        void* q8, void* k8, void* v8, float* sq, float* sk, float* sv,
+                        float* sv_max, float* k_mean, void* workspace, size_t workspace_bytes,
+                        void* cuda_stream) {
+  fqa_status st = check_shape(B, H, N, d, kQBlock);
+  if (st != FQA_OK) return st;
+  const void* ptrs[] = {q, k, v, q8, k8, v8, sq, sk, sv, sv_max, k_mean, workspace};
+  for (const void* p : ptrs)
+    if (p == nullptr) return FQA_ERR_INVALID_ARG;
+  if (workspace_bytes < fqa_quantize_workspace_bytes(B, H, N, d)) return FQA_ERR_INVALID_ARG;
+  const void* a16[] = {q, k, v, q8, k8, v8, workspace};
+  for (const void* p : a16)
+    if (!aligned(p, 16)) return FQA_ERR_MISALIGNED;
+  const void* a4[] = {sq, sk, sv, sv_max, k_mean};
+  for (const void* p : a4)
+    if (!aligned(p, 4)) return FQA_ERR_MISALIGNED;
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  float* partial = static_cast<float*>(workspace);
+  dim3 grid(N / kQBlock, H, B);
+  kmean_partial_kernel<<<grid, 128, 0, s>>>(static_cast<const __nv_bfloat16*>(k), partial, H, N);
+  kmean_reduce_kernel<<<B * H, 128, 0, s>>>(partial, k_mean, sv_max, N);
+  quantize_qkv_kernel<<<grid, 256, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+      static_cast<const __nv_bfloat16*>(v), k_mean, static_cast<uint8_t*>(q8),
+      static_cast<uint8_t*>(k8), static_cast<uint8_t*>(v8), sq, sk, sv, sv_max, H, N);
+  return launch_status();
+}
+
+static fqa_status check_attention_common(int B, int H, int N, int d, float softmax_scale,
+                                         void* out, fqa_out_dtype out_dtype) {
+  fqa_status st = check_shape(B, H, N, d, kBlockN);
+  if (st != FQA_OK) return st;
+  if (!(std::isfinite(softmax_scale) && softmax_scale > 0.0f)) return FQA_ERR_INVALID_ARG;
+  if (out == nullptr) return FQA_ERR_INVALID_ARG;
+  if (out_dtype != FQA_OUT_BF16 && out_dtype != FQA_OUT_F32) return FQA_ERR_INVALID_ARG;
+  if (!aligned(out, 16)) return FQA_ERR_MISALIGNED;
+  return FQA_OK;
+}
+
+fqa_status fqa_attention_fp8(const void* q8, const void* k8, const void* v8, const float* sq,
+                             const float* sk, const float* sv, const float* sv_max, int B, int H,
+                             int N, int d, float softmax_scale, void* out,
+                             fqa_out_dtype out_dtype, void* cuda_stream) {
+  fqa_status st = check_attention_common(B, H, N, d, softmax_scale, out, out_dtype);
+  if (st != FQA_OK) return st;
+  const void* ptrs[] = {q8, k8, v8, sq, sk, sv, sv_max};
+  for (const void* p : ptrs)
+    if (p == nullptr) return FQA_ERR_INVALID_ARG;
+  const void* a16[] = {q8, k8, v8};
+  for (const void* p : a16)
+    if (!aligned(p, 16)) return FQA_ERR_MISALIGNED;
+  const void* a4[] = {sq, sk, sv, sv_max};
+  for (const void* p : a4)
+    if (!aligned(p, 4)) return FQA_ERR_MISALIGNED;
+  uint32_t* status = status_ptr(&st);
+  if (!status) return st;
+  AttnParams prm{B, H, N, softmax_scale, sq, sk, sv, sv_max, out, out_dtype == FQA_OUT_F32, status};
+  return launch_attention<true>(q8, k8, v8, prm, static_cast<cudaStream_t>(cuda_stream));
+}
+
+fqa_status fqa_attention_bf16(const void* q, const void* k, const void* v, int B, int H, int N,
+                              int d, float softmax_scale, void* out, fqa_out_dtype out_dtype,
+                              void* cuda_stream) {
+  fqa_status st = check_attention_common(B, H, N, d, softmax_scale, out, out_dtype);
+  if (st != FQA_OK) return st;
+  const void* ptrs[] = {q, k, v};
+  for (const void* p : ptrs) {
+    if (p == nullptr) return FQA_ERR_INVALID_ARG;
+    if (!aligned(p, 16)) return FQA_ERR_MISALIGNED;
+  }
+  uint32_t* status = status_ptr(&st);
+  if (!status) return st;
+  AttnParams prm{B, H, N, softmax_scale, nullptr, nullptr, nullptr, nullptr, out,
+                 out_dtype == FQA_OUT_F32, status};
+  return launch_attention<false>(q, k, v, prm, static_cast<cudaStream_t>(cuda_stream));
+}
+
+fqa_status fqa_e4m3_encode(const float* x, uint8_t* out, size_t n, void* cuda_stream) {
+  if (x == nullptr || out == nullptr) return FQA_ERR_INVALID_ARG;
+  if (n == 0) return FQA_OK;
+  if (!aligned(x, 4)) return FQA_ERR_MISALIGNED;
+  e4m3_encode_kernel<<<148 * 8, 256, 0, static_cast<cudaStream_t>(cuda_stream)>>>(x, out, n);
+  return launch_status();
+}
+
+fqa_status fqa_debug_status(void* cuda_stream, uint32_t* flags_out) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess)
+    return FQA_ERR_CUDA;
+  uint32_t v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status_word, sizeof(v)) != cudaSuccess) return FQA_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_status_word, &zero, sizeof(zero)) != cudaSuccess) return FQA_ERR_CUDA;
+  if (flags_out) *flags_out = v;
+  return (v & kStatusTimeout) ? FQA_ERR_TIMEOUT : FQA_OK;
+}
+
+}  // extern "C"

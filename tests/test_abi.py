@@ -1,0 +1,104 @@
+"""The C ABI without a GPU: the library loads, exports every function that
+include/fqa.h declares, and rejects bad arguments on the host before any CUDA
+call (only argument sets that fail validation are used here)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from quantized_fp8_attention_b200 import build
+    build.build()
+    import quantized_fp8_attention_b200 as fqa
+    return fqa.lib()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "fqa.h")).read()
+    return sorted(set(re.findall(r"FQA_API\s+[\w\s\*]+?\b(fqa_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_path():
+    names = declared_functions()
+    for n in ("fqa_quantize", "fqa_attention_fp8", "fqa_attention_bf16", "fqa_quantize_workspace_bytes",
+              "fqa_status_string", "fqa_debug_status"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    for n in declared_functions():
+        assert hasattr(L, n), n
+
+
+def test_status_strings_and_version(L):
+    import quantized_fp8_attention_b200 as fqa
+    assert fqa.version() >> 16 == 1
+    assert [fqa.status_string(i) for i in range(6)] == [
+        "FQA_OK", "FQA_ERR_INVALID_ARG", "FQA_ERR_UNSUPPORTED", "FQA_ERR_MISALIGNED", "FQA_ERR_CUDA",
+        "FQA_ERR_TIMEOUT"]
+
+
+def test_workspace_bytes(L):
+    import quantized_fp8_attention_b200 as fqa
+    assert fqa.fqa_quantize_workspace_bytes(1, 24, 8704) == 24 * 136 * 128 * 4
+    assert fqa.fqa_quantize_workspace_bytes(2, 24, 16896) == 2 * 24 * 264 * 128 * 4
+    assert fqa.fqa_quantize_workspace_bytes(1, 1, 100) == 0       # N % 64 != 0
+    assert fqa.fqa_quantize_workspace_bytes(1, 1, 128, 64) == 0   # d != 128
+
+
+P = ctypes.c_void_p
+
+
+def _p(addr):
+    return P(addr)
+
+
+def test_quantize_validation(L):
+    ok = _p(0x10000)
+    args = lambda **kw: [kw.get(n, ok) for n in ("q", "k", "v")] + [
+        kw.get("B", 1), kw.get("H", 1), kw.get("N", 128), kw.get("d", 128)] + [
+        kw.get(n, ok) for n in ("q8", "k8", "v8", "sq", "sk", "sv", "svm", "km", "ws")] + [
+        kw.get("wsb", 1 << 20), None]
+    assert L.fqa_quantize(*args(q=None)) == 1
+    assert L.fqa_quantize(*args(ws=None)) == 1
+    assert L.fqa_quantize(*args(B=0)) == 1
+    assert L.fqa_quantize(*args(d=64)) == 2
+    assert L.fqa_quantize(*args(N=96)) == 2
+    assert L.fqa_quantize(*args(N=65600)) == 2
+    assert L.fqa_quantize(*args(B=300, H=300)) == 2
+    assert L.fqa_quantize(*args(wsb=16)) == 1
+    assert L.fqa_quantize(*args(k=_p(0x10008))) == 3
+    assert L.fqa_quantize(*args(sq=_p(0x10002))) == 3
+
+
+def test_attention_validation(L):
+    ok = _p(0x10000)
+    f = ctypes.c_float
+
+    def fp8(**kw):
+        return L.fqa_attention_fp8(*[kw.get(n, ok) for n in ("q8", "k8", "v8", "sq", "sk", "sv", "svm")],
+                                   kw.get("B", 1), kw.get("H", 1), kw.get("N", 128), kw.get("d", 128),
+                                   f(kw.get("scale", 0.088)), kw.get("out", ok), kw.get("dt", 0), None)
+
+    assert fp8(q8=None) == 1
+    assert fp8(out=None) == 1
+    assert fp8(scale=0.0) == 1
+    assert fp8(scale=float("inf")) == 1
+    assert fp8(dt=5) == 1
+    assert fp8(N=64) == 2
+    assert fp8(d=256) == 2
+    assert fp8(v8=_p(0x10001)) == 3
+    assert fp8(out=_p(0x10004)) == 3
+    bf = lambda **kw: L.fqa_attention_bf16(kw.get("q", ok), ok, ok, 1, 1, kw.get("N", 128), 128,
+                                           f(kw.get("scale", 0.088)), kw.get("out", ok), 0, None)
+    assert bf(q=None) == 1
+    assert bf(N=200) == 2
+    assert bf(scale=-1.0) == 1
+    assert bf(q=_p(0x10002)) == 3
+    assert L.fqa_e4m3_encode(None, ok, 4, None) == 1

@@ -1,0 +1,184 @@
+"""fqa_attention_fp8 / fqa_attention_bf16 on the GPU against the oracle.
+
+FP8 path, per workload (full tensors on the GPU, in the launch configuration
+the benchmark times; all rows checked on the two small workloads, sampled
+heads x rows [0,128) u [N/2,N/2+128) u [N-128,N) against all keys on the
+large ones):
+  (i)  FP32 verification output vs the oracle's binary64 output:
+       max abs <= 1e-2 and mean relative error <= 2e-3;
+  (ii) BF16 output vs the oracle's output rounded once to BF16: mean relative
+       error <= 2e-3 and every element within max(1e-2, one BF16 ulp of ref);
+  (iii) cosine vs exact unquantized FP64 attention, reported; it must not fall
+       more than 1e-3 below the oracle's own (the scheme's ceiling), and must
+       reach 0.995 where the oracle does.
+BF16 path: vs exact FP64 attention, cos >= 0.9999, mean rel <= 1e-2, FP32
+output within 2e-2 + 2^-8 |ref| elementwise.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import fqa_synth as synth
+import oracle
+from tests import gpu_util as U
+
+pytestmark = pytest.mark.gpu
+
+
+def _fqa():
+    import quantized_fp8_attention_b200 as fqa
+    return fqa
+
+
+def _rows_heads(w):
+    if w.B * w.H * w.N <= 24 * 1280:
+        return None, None
+    return U.sample_heads(w), U.sample_rows(w.N)
+
+
+def _pick(a: np.ndarray, heads, rows):
+    """[B,H,N,d] -> [n_heads, n_rows, d] in the oracle's order."""
+    if heads is None:
+        return a.reshape(-1, a.shape[2], a.shape[3])
+    return np.stack([a[b, h][rows] for (b, h) in heads])
+
+
+@pytest.mark.parametrize("idx", [0, 1, 2, 3, 4])
+def test_fp8_attention_matches_oracle(idx):
+    fqa = _fqa()
+    w = synth.workload(idx)
+    g = U.host_inputs(idx)
+    q, k, v = (U.to_device(g[t]) for t in "qkv")
+    qz = fqa.quantize(q, k, v)
+    out32 = fqa.attention_fp8(qz, U.SCALE, fqa.FQA_OUT_F32)
+    out16 = fqa.attention_fp8(qz, U.SCALE, fqa.FQA_OUT_BF16)
+    torch.cuda.synchronize()
+    assert fqa.fqa_debug_status()[0] == fqa.FQA_OK
+    heads, rows = _rows_heads(w)
+    ref = oracle.attention_fp8(U.oracle_quant(idx), U.SCALE, heads=heads, rows=rows)
+    got32 = _pick(out32.cpu().numpy(), heads, rows)
+    m = U.metrics(got32, ref)
+    print(f"\n[{w.name}] fp32 out vs oracle: {m}")
+    assert m["max_abs"] <= 1e-2 and m["mean_rel"] <= 2e-3, m
+    # (ii) production BF16 output
+    got16 = U.bf16_bits_to_f64(_pick(out16.view(torch.int16).cpu().numpy().view(np.uint16), heads, rows))
+    ref16 = U.bf16_bits_to_f64(oracle.bf16_round(ref))
+    m16 = U.metrics(got16, ref16)
+    print(f"[{w.name}] bf16 out vs oracle(bf16): {m16}")
+    assert m16["mean_rel"] <= 2e-3, m16
+    assert np.all(np.abs(got16 - ref16) <= np.maximum(1e-2, U.bf16_ulp(ref16)) + 1e-12)
+    # the BF16 output is the FP32 output rounded once to nearest even
+    b16 = out16.view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.array_equal(b16, oracle.bf16_round(out32.cpu().numpy().astype(np.float64)))
+    # (iii) accuracy against exact attention
+    ex = oracle.attention_exact(g["q"], g["k"], g["v"], U.SCALE, heads=heads, rows=rows)
+    cos_gpu = U.metrics(got32, ex)["cos"]
+    cos_orc = U.metrics(ref, ex)["cos"]
+    print(f"[{w.name}] cos vs exact FP64: gpu {cos_gpu:.6f}  oracle {cos_orc:.6f}")
+    assert cos_gpu >= cos_orc - 1e-3
+    if cos_orc >= 0.995:
+        assert cos_gpu >= 0.995
+
+
+@pytest.mark.parametrize("idx", [0, 1, 3])
+def test_bf16_attention_matches_exact(idx):
+    fqa = _fqa()
+    w = synth.workload(idx)
+    g = U.host_inputs(idx)
+    q, k, v = (U.to_device(g[t]) for t in "qkv")
+    out32 = fqa.attention_bf16(q, k, v, U.SCALE, fqa.FQA_OUT_F32)
+    out16 = fqa.attention_bf16(q, k, v, U.SCALE, fqa.FQA_OUT_BF16)
+    torch.cuda.synchronize()
+    assert fqa.fqa_debug_status()[0] == fqa.FQA_OK
+    heads, rows = _rows_heads(w)
+    ex = oracle.attention_exact(g["q"], g["k"], g["v"], U.SCALE, heads=heads, rows=rows)
+    got = _pick(out32.cpu().numpy(), heads, rows)
+    m = U.metrics(got, ex)
+    print(f"\n[{w.name}] bf16 path fp32 out vs exact: {m}")
+    assert m["cos"] >= 0.9999 and m["mean_rel"] <= 1e-2, m
+    assert np.all(np.abs(got - ex) <= 2e-2 + 2.0 ** -8 * np.abs(ex))
+    b16 = out16.view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.array_equal(b16, oracle.bf16_round(out32.cpu().numpy().astype(np.float64)))
+
+
+def _gen(shape, seed, scale=1.0):
+    rng = np.random.default_rng(seed)
+    return synth.round_to_bf16_bits(rng.standard_normal(shape) * scale)
+
+
+@pytest.mark.parametrize("N", [128, 256, 384])
+def test_fp8_small_sequences_all_rows(N):
+    """Single-tile and few-tile sequences, B*H = 3 heads, every row."""
+    fqa = _fqa()
+    shape = (1, 3, N, 128)
+    bits = {t: _gen(shape, 20 + i, 2.0) for i, t in enumerate("qkv")}
+    q, k, v = (U.to_device(bits[t]) for t in "qkv")
+    out = fqa.attention_fp8(fqa.quantize(q, k, v), U.SCALE, fqa.FQA_OUT_F32).cpu().numpy()
+    ref = oracle.attention_fp8(oracle.quantize(bits["q"], bits["k"], bits["v"]), U.SCALE)
+    m = U.metrics(out.reshape(ref.shape), ref)
+    assert m["max_abs"] <= 1e-2 and m["mean_rel"] <= 2e-3, m
+
+
+def test_fp8_uniform_scores_give_mean_of_v():
+    """Q = 0: every score is 0; with V made of one repeated 64 x 128 block all
+    V scales are equal, P = 448 exactly, and the output is the mean of the
+    dequantized V rows."""
+    fqa = _fqa()
+    rng = np.random.default_rng(30)
+    blk = rng.standard_normal((64, 128))
+    vb = synth.round_to_bf16_bits(np.tile(blk, (4, 1)).reshape(1, 1, 256, 128))
+    kb = _gen((1, 1, 256, 128), 31)
+    qb = np.zeros_like(kb)
+    out = fqa.attention_fp8(fqa.quantize(*(U.to_device(x) for x in (qb, kb, vb))), U.SCALE,
+                            fqa.FQA_OUT_F32).cpu().numpy()[0, 0]
+    qz = oracle.quantize(qb, kb, vb)
+    deq = oracle.e4m3_decode(qz["v8"][0, 0]) * np.repeat(qz["sv"][0, 0].astype(np.float64), 64)[:, None]
+    assert np.max(np.abs(out - deq.mean(axis=0)[None, :])) < 1e-5
+
+
+def test_fp8_zero_v_gives_zero():
+    fqa = _fqa()
+    qb, kb = _gen((1, 1, 256, 128), 40), _gen((1, 1, 256, 128), 41)
+    vb = np.zeros_like(qb)
+    out = fqa.attention_fp8(fqa.quantize(*(U.to_device(x) for x in (qb, kb, vb))), U.SCALE,
+                            fqa.FQA_OUT_F32)
+    assert torch.count_nonzero(out).item() == 0
+
+
+def test_fp8_longest_sequence_sampled():
+    """N = 65536 (the v1 maximum), one head, sampled rows against all keys."""
+    fqa = _fqa()
+    N = 65536
+    bits = {t: _gen((1, 1, N, 128), 50 + i) for i, t in enumerate("qkv")}
+    q, k, v = (U.to_device(bits[t]) for t in "qkv")
+    out = fqa.attention_fp8(fqa.quantize(q, k, v), U.SCALE, fqa.FQA_OUT_F32).cpu().numpy()
+    rows = [0, 1, 63, 64, 127, 128, N // 2, N - 129, N - 64, N - 1]
+    ref = oracle.attention_fp8(oracle.quantize(bits["q"], bits["k"], bits["v"]), U.SCALE, rows=rows)[0]
+    m = U.metrics(out[0, 0][rows], ref)
+    assert m["max_abs"] <= 1e-2 and m["mean_rel"] <= 2e-3, m
+
+
+def test_fp8_deterministic():
+    fqa = _fqa()
+    g = U.host_inputs(1)
+    q, k, v = (U.to_device(g[t]) for t in "qkv")
+    qz = fqa.quantize(q, k, v)
+    a = fqa.attention_fp8(qz, U.SCALE)
+    b = fqa.attention_fp8(qz, U.SCALE)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_attention_rejects_bad_arguments():
+    fqa = _fqa()
+    t = torch.zeros(1, 1, 192, 128, dtype=torch.uint8, device="cuda")   # N % 128 != 0
+    s = torch.ones(1, 1, 3, device="cuda")
+    sm = torch.ones(1, 1, device="cuda")
+    out = torch.empty(1, 1, 192, 128, dtype=torch.bfloat16, device="cuda")
+    assert fqa.fqa_attention_fp8(t, t, t, s, s, s, sm, U.SCALE, out, 0) == fqa.FQA_ERR_UNSUPPORTED
+    t = torch.zeros(1, 1, 128, 128, dtype=torch.uint8, device="cuda")
+    out = torch.empty(1, 1, 128, 128, dtype=torch.bfloat16, device="cuda")
+    assert fqa.fqa_attention_fp8(t, t, t, s, s, s, sm, float("nan"), out, 0) == fqa.FQA_ERR_INVALID_ARG
+    assert fqa.fqa_attention_fp8(t, t, t, s, s, s, sm, U.SCALE, out, 7) == fqa.FQA_ERR_INVALID_ARG
+    tb = torch.zeros(1, 1, 128, 128, dtype=torch.bfloat16, device="cuda")
+    assert fqa.fqa_attention_bf16(tb, tb, tb, -1.0, out, 0) == fqa.FQA_ERR_INVALID_ARG
