@@ -1,0 +1,369 @@
+"""Benchmark of the FP8 attention path on B200.
+
+One step = the whole FP8 hot path over one batch of synthetic input:
+fqa_quantize (K mean, Q/K/V block quantization) + fqa_attention_fp8, on the
+context-image editing workload (B=1, H=24, N=8704 = 512 text + 4096 context
+image + 4096 output image tokens, d=128).  value = 4*B*H*N^2*d FLOPs per step
+/ device time per step, in TFLOP/s, summed over ranks (each rank runs its own
+independently seeded batch; no data-path collective: weak scaling).
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fqa|reference]
+For N > 1 launch with torch.distributed.run (one rank per GPU).
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import fqa_synth as synth  # noqa: E402
+
+METRIC = "FP8 attention TFLOP/s and % of B200 FP8 peak at N=8704, H=24, d=128"
+WORKLOAD = "kontext_n8704"
+NOMINAL_FP8_TFLOPS = 4500.0
+NOMINAL_BF16_TFLOPS = 2250.0
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["quantized_fp8_attention_b200/csrc/attention.cuh",
+                  "quantized_fp8_attention_b200/csrc/device.cuh"]
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK), "fallback"
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def traffic_per_launch():
+    """DRAM bytes per attention launch from the committed ncu summary, if it
+    was taken on the current kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", "attn_fp8_kontext_n8704_traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    if d.get("kernel_source_sha") != kernel_source_sha():
+        return None
+    return d.get("traffic_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        mhz, mx, reasons = [], [], set()
+        for line in (self.out or "").strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 7:
+                continue
+            try:
+                mhz.append(float(f[0]))
+                mx.append(float(f[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not mhz:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(mhz)}
+
+
+def host_inputs(w, rank: int):
+    """Seeded BF16 inputs; each rank draws its own batch (seed offset by rank)."""
+    import dataclasses
+    wr = dataclasses.replace(w, seed=w.seed + 7919 * rank) if rank else w
+    return synth.generate(wr), wr
+
+
+# ------------------------------------------------------------ CPU baseline
+
+def oracle_sample(w, g, heads, rows):
+    """Time the CPU oracle on a bounded sample: the quantizer on the sampled
+    heads (full sequence) plus FP8 attention for `rows` query rows of each
+    sampled head against all keys.  Returns (seconds, flops, threads)."""
+    import oracle
+    oracle.build()
+    sel = lambda a: np.ascontiguousarray(np.stack([a[b, h] for (b, h) in heads])[None])
+    q, k, v = (sel(g[t]) for t in "qkv")
+    t0 = time.perf_counter()
+    qz = oracle.quantize(q, k, v)
+    oracle.attention_fp8(qz, oracle.softmax_scale(), heads=[(0, i) for i in range(len(heads))],
+                         rows=rows)
+    dt = time.perf_counter() - t0
+    flops = 4 * len(heads) * len(rows) * w.N * w.d
+    return dt, flops, oracle.num_threads()
+
+
+def cpu_baseline(w, g):
+    rows = list(range(0, w.N, max(1, w.N // 1024)))[:1024]
+    heads = [(0, h) for h in range(min(w.H, 4))]
+    dt, flops, threads = oracle_sample(w, g, heads, rows)
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"{len(heads)} heads: quantizer over all {w.N} tokens + FP8 attention for "
+                      f"{len(rows)} strided query rows x all {w.N} keys ({dt:.1f} s)"}
+
+
+def run_reference(args, rank: int, world: int):
+    """The reference arm: the CPU oracle as it stands, on bounded samples of
+    the same workload, in the same metric and unit."""
+    if rank != 0:
+        return
+    w = synth.workload(args.workload)
+    g = synth.generate(w, heads=[(0, h) for h in range(2)])
+    rows = list(range(0, w.N, max(1, w.N // 256)))[:256]
+    heads = [(0, 0), (0, 1)]
+    for _ in range(args.warmup):
+        oracle_sample(w, g, heads, rows[:16])
+    times, flops, threads = [], 0, 1
+    for _ in range(args.steps):
+        dt, flops, threads = oracle_sample(w, g, heads, rows)
+        times.append(dt)
+    t = sum(times) / len(times)
+    value = flops / t / 1e12
+    sample = (f"per step: quantizer on 2 heads x {w.N} tokens + FP8 attention for {len(rows)} strided "
+              f"rows x {w.N} keys on each")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+# ------------------------------------------------------------- GPU arm
+
+def run_fqa(args, rank: int, world: int):
+    import torch
+    import torch.distributed as dist
+
+    import quantized_fp8_attention_b200 as fqa
+    from quantized_fp8_attention_b200 import build as fqa_build
+
+    fqa_build.build()
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w0 = synth.workload(args.workload)
+    g, w = host_inputs(w0, rank)
+    B, H, N, d = w.B, w.H, w.N, w.d
+    flops = w.flops
+    scale = fqa.softmax_scale(d)
+
+    def dev_tensor(bits):
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    q, k, v = (dev_tensor(g[t]) for t in "qkv")
+    qz = fqa.alloc_quantized(B, H, N, dev)
+    ws = fqa.alloc_workspace(B, H, N, dev)
+    out = torch.empty(B, H, N, d, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        fqa.quantize(q, k, v, out=qz, workspace=ws)
+        fqa.attention_fp8(qz, scale, fqa.FQA_OUT_BF16, out=out)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    st, flags = fqa.fqa_debug_status()
+    if st != fqa.FQA_OK:
+        raise RuntimeError(f"device status {flags:#x} after warm-up")
+
+    K = args.steps
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * K + 1)]
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        ev[0].record(stream)
+        for i in range(K):
+            fqa.quantize(q, k, v, out=qz, workspace=ws)
+            ev[2 * i + 1].record(stream)
+            fqa.attention_fp8(qz, scale, fqa.FQA_OUT_BF16, out=out)
+            ev[2 * i + 2].record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    total_ms = ev[0].elapsed_time(ev[2 * K])
+    quant_ms = sum(ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(K)) / K
+    attn_ms = sum(ev[2 * i + 1].elapsed_time(ev[2 * i + 2]) for i in range(K)) / K
+    st, flags = fqa.fqa_debug_status()
+    if st != fqa.FQA_OK:
+        raise RuntimeError(f"device status {flags:#x} after the timed steps")
+
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_per_step = float(t.item()) / K
+    value = flops * world / (ms_per_step * 1e-3) / 1e12
+
+    # BF16 comparison path (a9), same inputs
+    for _ in range(3):
+        fqa.attention_bf16(q, k, v, scale, fqa.FQA_OUT_BF16, out=out)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    Kb = max(1, K // 2)
+    e0.record(stream)
+    for _ in range(Kb):
+        fqa.attention_bf16(q, k, v, scale, fqa.FQA_OUT_BF16, out=out)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    bf16_ms = e0.elapsed_time(e1) / Kb
+
+    # end to end through the public API with host buffers
+    hq, hk, hv = (torch.from_numpy(g[t].view(np.int16)).view(torch.bfloat16).pin_memory() for t in "qkv")
+    hout = torch.empty(B, H, N, d, dtype=torch.bfloat16).pin_memory()
+    h2d = 3 * hq.numel() * hq.element_size()
+    d2h = hout.numel() * hout.element_size()
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        step()
+        hout.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    Ke = max(3, K // 4)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(Ke):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    te = torch.tensor([e0.elapsed_time(e1) / Ke], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_ms = float(te.item())
+
+    if rank != 0:
+        return
+    pk, pk_kind = peaks()
+    fp8_peak = 2.0 * pk["bf16_tflops"]            # FP8 dense = 2 x BF16 dense (nominal ratio)
+    bf16_peak = pk["bf16_tflops"]
+    attn_tflops = flops / (attn_ms * 1e-3) / 1e12
+    quant_bytes = 9 * B * H * N * d
+    quant_gbs = quant_bytes / (quant_ms * 1e-3) / 1e9
+    bf16_tflops = flops / (bf16_ms * 1e-3) / 1e12
+    tr = traffic_per_launch()
+    cpu = None
+    if not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, g)
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 (fp32 accumulate)",
+        "data": "synthetic (seeded, FLUX-style token mix; see fqa_synth)",
+        "config": {"workload": w.name, "B": B, "H": H, "N": N, "d": d,
+                   "n_text": w.n_text, "n_ctx": w.n_ctx, "n_img": w.n_img,
+                   "step": "fqa_quantize + fqa_attention_fp8",
+                   "l2": "inputs larger than L2 (BF16 Q,K,V = %.0f MB per step)" % (3 * 2 * B * H * N * d / 1e6),
+                   "parallelism": f"dp{world} (independent batches)"},
+        "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<fp8>", "achieved": attn_tflops,
+                     "peak": fp8_peak, "unit": "TFLOP/s", "frac": attn_tflops / fp8_peak,
+                     "peak_source": f"{pk_kind}: 2 x bf16_tflops (burst) of MEASURED_PEAKS.json",
+                     "frac_of_nominal_4500": attn_tflops / NOMINAL_FP8_TFLOPS,
+                     "ms_per_launch": attn_ms, "traffic": tr},
+        "quantizer": {"ms": quant_ms, "gbs": quant_gbs, "algorithmic_bytes": quant_bytes,
+                      "frac_of_hbm": quant_gbs / pk["hbm_gbs"], "hbm_peak_gbs": pk["hbm_gbs"]},
+        "bf16_path": {"ms": bf16_ms, "tflops": bf16_tflops, "frac_of_bf16_peak": bf16_tflops / bf16_peak,
+                      "frac_of_nominal_2250": bf16_tflops / NOMINAL_BF16_TFLOPS},
+        "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": 4 * K,
+        "clocks": clk.summary(),
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="fqa", choices=["fqa", "reference"])
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_fqa(args, rank, world)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

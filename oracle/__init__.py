@@ -63,9 +63,9 @@ def lib():
         L.orc_k_mean.argtypes = [P, i, i, i, i, P]
         L.orc_quantize.argtypes = [P, P, P, i, i, i, i, P, P, P, P, P, P, P, P]
         L.orc_attention_core.argtypes = [P, P, P, P, P, P, ctypes.c_float, i, i,
-                                         ctypes.c_double, i, i, P, i, P]
+                                         ctypes.c_double, i, i, P, i, P, P, P]
         L.orc_attention_fp8.argtypes = [P, P, P, P, P, P, P, i, i, i, i, ctypes.c_float, i,
-                                        P, i, P, i, P]
+                                        P, i, P, i, P, P, P]
         L.orc_attention_exact.argtypes = [P, P, P, i, i, i, i, ctypes.c_double, P, i, P, i, P]
         L.orc_e4m3_encode_f32_array.argtypes = [P, ctypes.c_size_t, P]
         L.orc_bf16_round_array.argtypes = [P, ctypes.c_size_t, P]
@@ -155,19 +155,28 @@ def _heads_rows(B, H, N, heads, rows):
     return ha, ra
 
 
-def attention_fp8(qz: dict, softmax_scale: float, heads=None, rows=None, bc: int = 128) -> np.ndarray:
-    """Quantized-math attention on quantize() outputs -> [n_heads, n_rows, d] binary64."""
+def attention_fp8(qz: dict, softmax_scale: float, heads=None, rows=None, bc: int = 128,
+                  with_ambiguity: bool = False):
+    """Quantized-math attention on quantize() outputs -> [n_heads, n_rows, d] binary64.
+
+    with_ambiguity: also return (amb [n_heads, n_rows, d], namb [n_heads, n_rows]):
+    the output range spanned by P codes that a binary32 evaluation may round
+    to the other neighbour of an E4M3 midpoint, and how many such codes."""
     B, H, N, d = qz["q8"].shape
     ha, ra = _heads_rows(B, H, N, heads, rows)
     out = np.empty((len(ha), len(ra), d), dtype=np.float64)
+    amb = np.empty_like(out) if with_ambiguity else None
+    namb = np.empty((len(ha), len(ra)), dtype=np.int32) if with_ambiguity else None
     lib().orc_attention_fp8(_p(qz["q8"]), _p(qz["k8"]), _p(qz["v8"]), _p(qz["sq"]),
                             _p(qz["sk"]), _p(qz["sv"]), _p(qz["sv_max"]), B, H, N, d,
                             float(np.float32(softmax_scale)), bc, _p(ha), len(ha), _p(ra),
-                            len(ra), _p(out))
-    return out
+                            len(ra), _p(out), None if amb is None else _p(amb),
+                            None if namb is None else _p(namb))
+    return (out, amb, namb) if with_ambiguity else out
 
 
-def attention_core(qc, kc, vc, sq, sk, sv, sv_max, scale, bc=128, quantize_p=True, rows=None):
+def attention_core(qc, kc, vc, sq, sk, sv, sv_max, scale, bc=128, quantize_p=True, rows=None,
+                   with_ambiguity=False):
     """The tiled core on binary64 operand values for one head ([N,d] each)."""
     qc = np.ascontiguousarray(qc, dtype=np.float64)
     kc = np.ascontiguousarray(kc, dtype=np.float64)
@@ -178,10 +187,13 @@ def attention_core(qc, kc, vc, sq, sk, sv, sv_max, scale, bc=128, quantize_p=Tru
     sv = np.ascontiguousarray(sv, dtype=np.float32)
     ra = np.ascontiguousarray(np.array(list(range(N) if rows is None else rows), dtype=np.int32))
     out = np.empty((len(ra), d), dtype=np.float64)
+    amb = np.empty_like(out) if with_ambiguity else None
+    namb = np.empty(len(ra), dtype=np.int32) if with_ambiguity else None
     lib().orc_attention_core(_p(qc), _p(kc), _p(vc), _p(sq), _p(sk), _p(sv), float(sv_max),
                              N, d, float(scale), bc, int(bool(quantize_p)), _p(ra), len(ra),
-                             _p(out))
-    return out
+                             _p(out), None if amb is None else _p(amb),
+                             None if namb is None else _p(namb))
+    return (out, amb, namb) if with_ambiguity else out
 
 
 def attention_exact(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float,

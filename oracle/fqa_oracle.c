@@ -210,11 +210,30 @@ void orc_quantize(const uint16_t *q, const uint16_t *k, const uint16_t *v,
  *   acc_c  = acc_c * 2^(m_{t-1} - m_t) + sum_j P_ij vc_jc
  *   O_ic   = acc_c * (sv_max / 448) / l
  * sv_max == 0 (V entirely zero) gives O = 0.
- * rows: the query rows of this head to evaluate; out: [n_rows, d]. */
+ * rows: the query rows of this head to evaluate; out: [n_rows, d].
+ * amb (optional, [n_rows, d]): bound on |O - O'| over every O' whose P codes
+ * differ from these only where a binary32 evaluation of p * 448 * rv can fall
+ * on the other side of an E4M3 rounding midpoint (see p_eval_bound); namb
+ * (optional, [n_rows]): how many P codes of the row are such. */
+/* Relative error bound of a binary32 evaluation of one P value p * 448 * rv
+ * (before E4M3 rounding), used to flag P codes that a kernel working in
+ * binary32 may legitimately round the other way.  Sources: the FP32
+ * accumulation of the 128 code products (2^-22 of their magnitude sum), the
+ * binary32 roundings of the score, its scale and the running maximum
+ * (2^-22 of |x| + 2|m|, in log2 units), the hardware exp2 approximation
+ * (2^-21 relative) and the final products (2^-22). */
+static double p_eval_bound(double abs_prod_sum, double a, double x, double m)
+{
+    const double LN2 = 0.69314718055994530942;
+    double dx = ldexp(a * abs_prod_sum + fabs(x) + 2.0 * fabs(m), -22);
+    return LN2 * dx + ldexp(1.0, -21) + ldexp(1.0, -22);
+}
+
 static void attention_core_head(const double *qc, const double *kc, const double *vc,
                                 const float *sq, const float *sk, const float *sv, float sv_max,
                                 int N, int d, double scale, int bc, int quantize_p,
-                                const int *rows, int n_rows, double *out)
+                                const int *rows, int n_rows, double *out,
+                                double *amb, int *namb)
 {
     const double LOG2E = 1.4426950408889634073599246810019;  /* log2(e) */
     #pragma omp parallel for schedule(dynamic, 4)
@@ -222,33 +241,61 @@ static void attention_core_head(const double *qc, const double *kc, const double
         int i = rows[r];
         double *o = out + (size_t)r * d;
         double *x = (double *)malloc(sizeof(double) * bc);
+        double *aps = (double *)malloc(sizeof(double) * bc);
         double *acc = (double *)calloc(d, sizeof(double));
+        double *aacc = (double *)calloc(d, sizeof(double));
         double m = -INFINITY, l = 0.0;
+        int n_amb = 0;
         if (sv_max == 0.0f) {
             for (int c = 0; c < d; c++) o[c] = 0.0;
-            free(x); free(acc);
+            if (amb) for (int c = 0; c < d; c++) amb[(size_t)r * d + c] = 0.0;
+            if (namb) namb[r] = 0;
+            free(x); free(aps); free(acc); free(aacc);
             continue;
         }
         for (int t0 = 0; t0 < N; t0 += bc) {
             int t1 = t0 + bc < N ? t0 + bc : N;
             double tmax = -INFINITY;
             for (int j = t0; j < t1; j++) {
-                double s = 0.0;
-                for (int c = 0; c < d; c++)
-                    s += qc[(size_t)i * d + c] * kc[(size_t)j * d + c];
+                double s = 0.0, sa = 0.0;
+                for (int c = 0; c < d; c++) {
+                    double pr = qc[(size_t)i * d + c] * kc[(size_t)j * d + c];
+                    s += pr;
+                    sa += fabs(pr);
+                }
                 x[j - t0] = s * (double)sq[i / 64] * (double)sk[j / 64] * scale * LOG2E;
+                aps[j - t0] = sa;
                 if (x[j - t0] > tmax) tmax = x[j - t0];
             }
             double m_new = tmax > m ? tmax : m;
             double alpha = exp2(m - m_new);      /* 0 on the first tile */
             l *= alpha;
             for (int c = 0; c < d; c++) acc[c] *= alpha;
+            for (int c = 0; c < d; c++) aacc[c] *= alpha;
             for (int j = t0; j < t1; j++) {
                 double p = exp2(x[j - t0] - m_new);
                 double rv = (double)sv[j / 64] / (double)sv_max;
                 double P = p * 448.0 * rv;
-                if (quantize_p)
-                    P = orc_e4m3_decode(orc_e4m3_encode(P));
+                if (quantize_p) {
+                    double Pv = P;
+                    uint8_t code = orc_e4m3_encode(Pv);
+                    P = orc_e4m3_decode(code);
+                    if (amb || namb) {
+                        /* both neighbours of a rounding midpoint are valid codes
+                         * when the binary32 evaluation can cross it */
+                        double a = (double)sq[i / 64] * (double)sk[j / 64] * scale * LOG2E;
+                        double eta = p_eval_bound(aps[j - t0], a, x[j - t0], m_new);
+                        uint8_t lo = orc_e4m3_encode(Pv * (1.0 - eta));
+                        uint8_t hi = orc_e4m3_encode(Pv * (1.0 + eta));
+                        if (lo != code || hi != code) {
+                            double dP = fmax(fabs(orc_e4m3_decode(lo) - P),
+                                             fabs(orc_e4m3_decode(hi) - P));
+                            n_amb++;
+                            for (int c = 0; c < d; c++)
+                                aacc[c] += dP * fabs(vc[(size_t)j * d + c]);
+                        }
+                    }
+                }
                 l += p;
                 for (int c = 0; c < d; c++)
                     acc[c] += P * vc[(size_t)j * d + c];
@@ -257,8 +304,14 @@ static void attention_core_head(const double *qc, const double *kc, const double
         }
         for (int c = 0; c < d; c++)
             o[c] = acc[c] * ((double)sv_max / 448.0) / l;
+        if (amb)
+            for (int c = 0; c < d; c++)
+                amb[(size_t)r * d + c] = aacc[c] * ((double)sv_max / 448.0) / l;
+        if (namb) namb[r] = n_amb;
         free(x);
+        free(aps);
         free(acc);
+        free(aacc);
     }
 }
 
@@ -266,10 +319,10 @@ static void attention_core_head(const double *qc, const double *kc, const double
 void orc_attention_core(const double *qc, const double *kc, const double *vc,
                         const float *sq, const float *sk, const float *sv, float sv_max,
                         int N, int d, double scale, int bc, int quantize_p,
-                        const int *rows, int n_rows, double *out)
+                        const int *rows, int n_rows, double *out, double *amb, int *namb)
 {
     attention_core_head(qc, kc, vc, sq, sk, sv, sv_max, N, d, scale, bc, quantize_p,
-                        rows, n_rows, out);
+                        rows, n_rows, out, amb, namb);
 }
 
 /* FP8 attention on quantizer outputs (codes in natural [B,H,N,d] layout).
@@ -279,7 +332,7 @@ void orc_attention_fp8(const uint8_t *q8, const uint8_t *k8, const uint8_t *v8,
                        const float *sq, const float *sk, const float *sv, const float *sv_max,
                        int B, int H, int N, int d, float softmax_scale, int bc,
                        const int *heads, int n_heads, const int *rows, int n_rows,
-                       double *out)
+                       double *out, double *amb, int *namb)
 {
     int nblk = N / 64;
     (void)B;
@@ -299,7 +352,9 @@ void orc_attention_fp8(const uint8_t *q8, const uint8_t *k8, const uint8_t *v8,
         size_t sidx = ((size_t)b * H + h) * nblk;
         attention_core_head(qc, kc, vc, sq + sidx, sk + sidx, sv + sidx,
                             sv_max[(size_t)b * H + h], N, d, (double)softmax_scale, bc, 1,
-                            rows, n_rows, out + (size_t)hh * n_rows * d);
+                            rows, n_rows, out + (size_t)hh * n_rows * d,
+                            amb ? amb + (size_t)hh * n_rows * d : NULL,
+                            namb ? namb + (size_t)hh * n_rows : NULL);
     }
     free(qc); free(kc); free(vc);
 }

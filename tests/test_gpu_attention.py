@@ -5,9 +5,13 @@ the benchmark times; all rows checked on the two small workloads, sampled
 heads x rows [0,128) u [N/2,N/2+128) u [N-128,N) against all keys on the
 large ones):
   (i)  FP32 verification output vs the oracle's binary64 output:
-       max abs <= 1e-2 and mean relative error <= 2e-3;
+       mean relative error <= 2e-3 and every element within 1e-2 + amb, where
+       amb is the oracle's bound on what P codes lying within binary32
+       evaluation error of an E4M3 rounding midpoint can change (such a code
+       may round either way; elsewhere amb = 0 and the bound is 1e-2);
   (ii) BF16 output vs the oracle's output rounded once to BF16: mean relative
-       error <= 2e-3 and every element within max(1e-2, one BF16 ulp of ref);
+       error <= 2e-3 and every element within max(1e-2, one BF16 ulp of ref)
+       + amb;
   (iii) cosine vs exact unquantized FP64 attention, reported; it must not fall
        more than 1e-3 below the oracle's own (the scheme's ceiling), and must
        reach 0.995 where the oracle does.
@@ -56,18 +60,22 @@ def test_fp8_attention_matches_oracle(idx):
     torch.cuda.synchronize()
     assert fqa.fqa_debug_status()[0] == fqa.FQA_OK
     heads, rows = _rows_heads(w)
-    ref = oracle.attention_fp8(U.oracle_quant(idx), U.SCALE, heads=heads, rows=rows)
+    ref, amb, namb = oracle.attention_fp8(U.oracle_quant(idx), U.SCALE, heads=heads, rows=rows,
+                                          with_ambiguity=True)
     got32 = _pick(out32.cpu().numpy(), heads, rows)
     m = U.metrics(got32, ref)
-    print(f"\n[{w.name}] fp32 out vs oracle: {m}")
-    assert m["max_abs"] <= 1e-2 and m["mean_rel"] <= 2e-3, m
+    err = np.abs(got32 - ref)
+    print(f"\n[{w.name}] fp32 out vs oracle: {m}; ambiguous P codes {int(namb.sum())}, "
+          f"elements over 1e-2: {int((err > 1e-2).sum())} (all covered: {bool(np.all(err <= 1e-2 + amb))})")
+    assert m["mean_rel"] <= 2e-3, m
+    assert np.all(err <= 1e-2 + amb), float((err - amb).max())
     # (ii) production BF16 output
     got16 = U.bf16_bits_to_f64(_pick(out16.view(torch.int16).cpu().numpy().view(np.uint16), heads, rows))
     ref16 = U.bf16_bits_to_f64(oracle.bf16_round(ref))
     m16 = U.metrics(got16, ref16)
     print(f"[{w.name}] bf16 out vs oracle(bf16): {m16}")
     assert m16["mean_rel"] <= 2e-3, m16
-    assert np.all(np.abs(got16 - ref16) <= np.maximum(1e-2, U.bf16_ulp(ref16)) + 1e-12)
+    assert np.all(np.abs(got16 - ref16) <= np.maximum(1e-2, U.bf16_ulp(ref16)) + amb + 1e-12)
     # the BF16 output is the FP32 output rounded once to nearest even
     b16 = out16.view(torch.int16).cpu().numpy().view(np.uint16)
     assert np.array_equal(b16, oracle.bf16_round(out32.cpu().numpy().astype(np.float64)))
@@ -115,9 +123,11 @@ def test_fp8_small_sequences_all_rows(N):
     bits = {t: _gen(shape, 20 + i, 2.0) for i, t in enumerate("qkv")}
     q, k, v = (U.to_device(bits[t]) for t in "qkv")
     out = fqa.attention_fp8(fqa.quantize(q, k, v), U.SCALE, fqa.FQA_OUT_F32).cpu().numpy()
-    ref = oracle.attention_fp8(oracle.quantize(bits["q"], bits["k"], bits["v"]), U.SCALE)
+    ref, amb, _ = oracle.attention_fp8(oracle.quantize(bits["q"], bits["k"], bits["v"]), U.SCALE,
+                                       with_ambiguity=True)
     m = U.metrics(out.reshape(ref.shape), ref)
-    assert m["max_abs"] <= 1e-2 and m["mean_rel"] <= 2e-3, m
+    assert m["mean_rel"] <= 2e-3, m
+    assert np.all(np.abs(out.reshape(ref.shape) - ref) <= 1e-2 + amb)
 
 
 def test_fp8_uniform_scores_give_mean_of_v():
@@ -154,9 +164,11 @@ def test_fp8_longest_sequence_sampled():
     q, k, v = (U.to_device(bits[t]) for t in "qkv")
     out = fqa.attention_fp8(fqa.quantize(q, k, v), U.SCALE, fqa.FQA_OUT_F32).cpu().numpy()
     rows = [0, 1, 63, 64, 127, 128, N // 2, N - 129, N - 64, N - 1]
-    ref = oracle.attention_fp8(oracle.quantize(bits["q"], bits["k"], bits["v"]), U.SCALE, rows=rows)[0]
-    m = U.metrics(out[0, 0][rows], ref)
-    assert m["max_abs"] <= 1e-2 and m["mean_rel"] <= 2e-3, m
+    ref, amb, _ = oracle.attention_fp8(oracle.quantize(bits["q"], bits["k"], bits["v"]), U.SCALE,
+                                       rows=rows, with_ambiguity=True)
+    m = U.metrics(out[0, 0][rows], ref[0])
+    assert m["mean_rel"] <= 2e-3, m
+    assert np.all(np.abs(out[0, 0][rows] - ref[0]) <= 1e-2 + amb[0])
 
 
 def test_fp8_deterministic():

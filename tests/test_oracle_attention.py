@@ -140,13 +140,20 @@ def _golden_inputs(case):
     return qc, kc, vc
 
 
-@pytest.mark.parametrize("idx", [0, 1, 2])
+@pytest.mark.parametrize("idx", [0, 1, 2, 3])
 def test_hand_worked_p_rounding_cases(idx):
     case = json.load(open(GOLDEN))["cases"][idx]
     qc, kc, vc = _golden_inputs(case)
-    out = oracle.attention_core(qc, kc, vc, np.array(case["sq"], np.float32),
-                                np.array(case["sk"], np.float32), np.array(case["sv"], np.float32),
-                                case["sv_max"], LN2, bc=case["bc"], quantize_p=True, rows=[0])[0]
+    out, amb, namb = oracle.attention_core(
+        qc, kc, vc, np.array(case["sq"], np.float32), np.array(case["sk"], np.float32),
+        np.array(case["sv"], np.float32), case["sv_max"], LN2, bc=case["bc"], quantize_p=True,
+        rows=[0], with_ambiguity=True)
+    out, amb, namb = out[0], amb[0], int(namb[0])
+    exp_amb = np.zeros(128)
+    for c, val in case.get("expected_amb", {}).items():
+        exp_amb[int(c)] = val
+    assert namb == case.get("expected_namb", 0)
+    assert np.max(np.abs(amb - exp_amb)) < 1e-9
     l = eval(case["expected_l"], {"__builtins__": {}})
     if "expected_weights" in case:
         weights = [eval(wt, {"__builtins__": {}}) for wt in case["expected_weights"]]
@@ -167,3 +174,39 @@ def test_config0_quantized_close_to_exact():
     e = oracle.attention_exact(g["q"], g["k"], g["v"], sc)
     cos = float((a * e).sum() / np.sqrt((a * a).sum() * (e * e).sum()))
     assert cos > 0.995
+
+
+def test_ambiguity_bound_covers_binary32_evaluation():
+    """Re-evaluate the P codes of a workload head the way a binary32 kernel
+    does (scores, scales and the running max rounded to binary32, P values
+    rounded to binary32 before encoding): every code that differs from the
+    binary64 oracle's is one the oracle flagged, and the binary32 result lies
+    within the reported bound."""
+    w = s.workload(1)
+    g = s.generate(w, heads=[(0, 0)])
+    qz = oracle.quantize(g["q"][:, :1], g["k"][:, :1], g["v"][:, :1])
+    ref, amb, namb = oracle.attention_fp8(qz, oracle.softmax_scale(), with_ambiguity=True)
+    dec = oracle.e4m3_decode
+    qc, kc, vc = (dec(qz[t][0, 0]) for t in ("q8", "k8", "v8"))
+    sq, sk, sv = (qz[t][0, 0] for t in ("sq", "sk", "sv"))
+    svm = qz["sv_max"][0, 0]
+    c = np.float32(np.float32(oracle.softmax_scale()) * np.float32(1.4426950408889634))
+    a32 = (np.repeat(sq, 64)[:, None] * np.repeat((sk * c).astype(np.float32), 64)[None, :]).astype(np.float32)
+    x32 = ((qc @ kc.T).astype(np.float32) * a32).astype(np.float32)
+    cj = np.repeat((np.float32(448.0) * (sv / svm).astype(np.float32)).astype(np.float32), 64)
+    N = w.N
+    m = np.full(N, -np.inf, np.float32)
+    acc = np.zeros((N, 128))
+    l = np.zeros(N)
+    for t0 in range(0, N, 128):
+        sl = slice(t0, t0 + 128)
+        m_new = np.maximum(m, x32[:, sl].max(1))
+        alpha = np.exp2(m.astype(np.float64) - m_new)
+        p = np.exp2((x32[:, sl] - m_new[:, None]).astype(np.float32)).astype(np.float32)
+        P = dec(oracle.e4m3_encode((p * cj[None, sl]).astype(np.float32)))
+        acc = acc * alpha[:, None] + P @ vc[sl]
+        l = l * alpha + p.astype(np.float64).sum(1)
+        m = m_new
+    out32 = acc * (float(svm) / 448.0) / l[:, None]
+    # beyond flipped codes, binary32 scores shift O by ~1e-4 (alpha, l)
+    assert np.all(np.abs(out32 - ref[0]) <= amb[0] + 1e-3)
