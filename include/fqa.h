@@ -123,6 +123,38 @@ FQA_API fqa_status fqa_quantize(const void* q, const void* k, const void* v, int
                         void* cuda_stream);
 
 /*
+ * fqa_quantize_noalloc -- fqa_quantize() without a workspace argument, for
+ * callers that cannot allocate device memory at call time: for example an
+ * operator running inside a host framework that owns all device memory and
+ * forbids allocation while it executes, or a runtime whose device memory is
+ * planned once up front.  (The pages have no counterpart; this is a library
+ * convenience.)
+ *
+ * Same arguments, results and bit-exactness as fqa_quantize(), minus
+ * workspace/workspace_bytes.  The K-mean scratch is a fixed array of
+ * fqa_quantize_noalloc_max_workspace_bytes() = 8 MiB inside the library, one
+ * per GPU that loads it, held until the process exits.  Sizes whose scratch
+ * need, fqa_quantize_workspace_bytes(B,H,N,d), exceeds that limit are rejected
+ * with FQA_ERR_UNSUPPORTED before anything is launched.  Neither this call nor
+ * its set-up allocates device memory (no cudaMalloc, cudaFree or allocating
+ * library routine).
+ *
+ * The first call on a device looks up the device address of that device's
+ * array (once per device, with that device current); make that first call
+ * before any stream capture.  Every call on a device shares the one array and
+ * leaves its last contents there; nothing in it needs to start at zero.  Calls
+ * that overlap on the GPU (e.g. on two streams at once) race on the array:
+ * order them on one stream or synchronize between them.
+ */
+FQA_API fqa_status fqa_quantize_noalloc(const void* q, const void* k, const void* v, int B, int H,
+                                        int N, int d, void* q8, void* k8, void* v8, float* sq,
+                                        float* sk, float* sv, float* sv_max, float* k_mean,
+                                        void* cuda_stream);
+
+/* Size of the fixed scratch array fqa_quantize_noalloc() uses (8 MiB). */
+FQA_API size_t fqa_quantize_noalloc_max_workspace_bytes(void);
+
+/*
  * fqa_attention_fp8 -- fused FP8 attention on fqa_quantize() outputs.
  * [RTX-DE] Table-1 paragraph (attention in FP8); [RTX-KR] SDPA paragraph.
  *

@@ -107,6 +107,20 @@ def fqa_quantize(q, k, v, q8, k8, v8, sq, sk, sv, sv_max, k_mean, workspace, str
                              _stream(stream))
 
 
+def fqa_quantize_noalloc(q, k, v, q8, k8, v8, sq, sk, sv, sv_max, k_mean, stream=None) -> int:
+    """fqa_quantize without a workspace (for callers that cannot allocate
+    device memory when they call): the library keeps the scratch in a fixed
+    8 MiB array per GPU.  Returns the fqa_status code."""
+    L = _load()
+    f = L.fqa_quantize_noalloc
+    P, I = ctypes.c_void_p, ctypes.c_int
+    f.restype = I
+    f.argtypes = [P, P, P, I, I, I, I, P, P, P, P, P, P, P, P, P]
+    B, H, N, d = q.shape
+    return f(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, _ptr(q8), _ptr(k8), _ptr(v8), _ptr(sq),
+             _ptr(sk), _ptr(sv), _ptr(sv_max), _ptr(k_mean), _stream(stream))
+
+
 def fqa_attention_fp8(q8, k8, v8, sq, sk, sv, sv_max, softmax_scale, out, out_dtype, stream=None) -> int:
     B, H, N, d = q8.shape
     return _load().fqa_attention_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(sq), _ptr(sk), _ptr(sv),

@@ -237,3 +237,63 @@ fqa_status fqa_debug_status(void* cuda_stream, uint32_t* flags_out) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// fqa_quantize_noalloc: fqa_quantize for callers that cannot allocate device
+// memory when they call.  The K-mean partial sums live in a fixed array inside
+// the library instead of a caller-provided workspace.
+namespace fqa {
+
+// Upper bound of the scratch the quantizer needs, B*H*(N/64)*128*4 bytes:
+// 8 MiB covers B*H*(N/64) <= 16384 (e.g. B=2, H=24, N=16896 needs 6.2 MiB).
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;
+
+// One copy per GPU that loads the library, held until the process exits.
+// In host code this name is only a stand-in: the device address comes from
+// cudaGetSymbolAddress below.
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
+
+struct NoAllocCache {
+  std::once_flag once;
+  float* ptr = nullptr;
+  cudaError_t err = cudaSuccess;
+};
+NoAllocCache g_noalloc[kMaxDevices];
+
+// Device address of this device's scratch array, looked up once per device
+// with that device current.
+static float* noalloc_scratch(fqa_status* st) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    *st = FQA_ERR_CUDA;
+    return nullptr;
+  }
+  NoAllocCache& c = g_noalloc[dev];
+  std::call_once(c.once, [&c]() {
+    void* p = nullptr;
+    c.err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (c.err == cudaSuccess) c.ptr = static_cast<float*>(p);
+  });
+  if (c.err != cudaSuccess || c.ptr == nullptr) {
+    *st = FQA_ERR_CUDA;
+    return nullptr;
+  }
+  return c.ptr;
+}
+
+}  // namespace fqa
+
+extern "C" size_t fqa_quantize_noalloc_max_workspace_bytes(void) { return kNoAllocScratchBytes; }
+
+extern "C" fqa_status fqa_quantize_noalloc(const void* q, const void* k, const void* v, int B, int H,
+                                           int N, int d, void* q8, void* k8, void* v8, float* sq,
+                                           float* sk, float* sv, float* sv_max, float* k_mean,
+                                           void* cuda_stream) {
+  fqa_status st = check_shape(B, H, N, d, kQBlock);
+  if (st != FQA_OK) return st;
+  if (fqa_quantize_workspace_bytes(B, H, N, d) > kNoAllocScratchBytes) return FQA_ERR_UNSUPPORTED;
+  float* scratch = noalloc_scratch(&st);
+  if (scratch == nullptr) return st;
+  return fqa_quantize(q, k, v, B, H, N, d, q8, k8, v8, sq, sk, sv, sv_max, k_mean, scratch,
+                      kNoAllocScratchBytes, cuda_stream);
+}
