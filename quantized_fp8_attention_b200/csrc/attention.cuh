@@ -40,6 +40,26 @@ constexpr int kBlockN = 128;   // keys per KV tile (part of the FP8 rounding rul
 constexpr int kAttnThreads = 192;
 constexpr int kMaxScaleBlocks = 1024;   // N <= 65536
 
+// Of every 8 exponentials (pairs of keys) this many are evaluated by the FMA
+// pipe polynomial instead of the MUFU ex2 unit, to balance the two pipes.
+#ifndef FQA_EXP2_POLY_PER8
+#define FQA_EXP2_POLY_PER8 0
+#endif
+constexpr int kPolyPer8 = FQA_EXP2_POLY_PER8;
+
+// p for two keys at once: 2^(x - m) with x = fl(S * a) already rounded and
+// m = max x.  x - m is exact near the maximum (Sterbenz), so the row maximum
+// gets p = 1 exactly and the row sum l carries no common rounding factor (a
+// fused S * a - m would give the maximum p = 2^delta, delta the rounding
+// residue of m, and bias l by ~|m| 2^-24).  The subtraction is written as
+// fma(x, 1, -m) so that the multiply producing x can never be fused into it.
+template <bool kPoly>
+__device__ __forceinline__ float2 exp2_pair(float2 x, float2 nm2) {
+  const float2 d = f2_fma(x, make_float2(1.0f, 1.0f), nm2);
+  if constexpr (kPoly) return exp2_poly2(d);
+  return make_float2(ex2_approx(d.x), ex2_approx(d.y));
+}
+
 struct AttnParams {
   int B, H, N;
   float softmax_scale;
@@ -253,10 +273,7 @@ __global__ void __launch_bounds__(kAttnThreads, kFP8 ? 2 : 1)
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(tS + lane_off + 32u * c, sr[c]);
       tmem_wait_ld();
-      float x[128];
-#pragma unroll
-      for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(sr[c >> 5][c & 31]);
-      // scores in log2 units, rounded once: x = fl(S * a)
+      // scores in log2 units, rounded once: x = fl(S * a) (per 64-key block scale)
       float a0, a1;
       if constexpr (kFP8) {
         a0 = a_row * skc[2 * j];
@@ -264,52 +281,83 @@ __global__ void __launch_bounds__(kAttnThreads, kFP8 ? 2 : 1)
       } else {
         a0 = a1 = c_log2e;
       }
-      float tmax = -INFINITY;
+      float2 X[64];
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        x[c] = x[c] * (c < 64 ? a0 : a1);
-        tmax = fmaxf(tmax, x[c]);
+      for (int e = 0; e < 64; ++e) {
+        const float a = (e < 32) ? a0 : a1;
+        X[e] = f2_mul(make_float2(__uint_as_float(sr[e >> 4][(2 * e) & 31]),
+                                  __uint_as_float(sr[e >> 4][(2 * e + 1) & 31])),
+                      make_float2(a, a));
       }
+      // tile max of x: 4 independent chains of 3-input maxima over 16 pairs each
+      float cm[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        cm[r] = fmaxf(X[16 * r].x, X[16 * r].y);
+#pragma unroll
+        for (int t = 1; t < 16; ++t) cm[r] = fmax3(cm[r], X[16 * r + t].x, X[16 * r + t].y);
+      }
+      const float tmax = fmaxf(fmax3(cm[0], cm[1], cm[2]), cm[3]);
       const float m_new = fmaxf(m, tmax);
       const float alpha = ex2_approx(m - m_new);     // 0 on the first tile
       // O correction: rescale the accumulated rows whose max moved.  The
       // barS phase we waited on completes after the previous P.V MMA.
       if (j > 0 && __any_sync(0xffffffffu, m_new != m)) {
+        const float2 al2 = make_float2(alpha, alpha);
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t o[32];
           tmem_ld32(tO + lane_off + 32u * c, o);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          for (int e = 0; e < 32; e += 2) {
+            float2 v = f2_mul(make_float2(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), al2);
+            o[e] = __float_as_uint(v.x);
+            o[e + 1] = __float_as_uint(v.y);
+          }
           tmem_st32(tO + lane_off + 32u * c, o);
         }
       }
-      float lsum = 0.0f;
+      const float2 nm2 = make_float2(-m_new, -m_new);
+      float2 l2 = make_float2(0.0f, 0.0f);
       if constexpr (kFP8) {
-        const float c0 = pvc[2 * j], c1 = pvc[2 * j + 1];
         uint32_t pw[32];
 #pragma unroll
+        const float c0 = pvc[2 * j], c1 = pvc[2 * j + 1];
+#pragma unroll
         for (int w = 0; w < 32; ++w) {
-          float e0 = ex2_approx(x[4 * w] - m_new), e1 = ex2_approx(x[4 * w + 1] - m_new);
-          float e2 = ex2_approx(x[4 * w + 2] - m_new), e3 = ex2_approx(x[4 * w + 3] - m_new);
-          lsum += (e0 + e1) + (e2 + e3);
           const float cc = (w < 16) ? c0 : c1;
-          pw[w] = e4m3x2(e0 * cc, e1 * cc) | (e4m3x2(e2 * cc, e3 * cc) << 16);
+          const float2 c2 = make_float2(cc, cc);
+          float2 p01, p23;
+          if ((w % 4) < kPolyPer8 / 2) {
+            p01 = exp2_pair<true>(X[2 * w], nm2);
+            p23 = exp2_pair<true>(X[2 * w + 1], nm2);
+          } else if ((w % 4) == kPolyPer8 / 2 && (kPolyPer8 & 1)) {
+            p01 = exp2_pair<true>(X[2 * w], nm2);
+            p23 = exp2_pair<false>(X[2 * w + 1], nm2);
+          } else {
+            p01 = exp2_pair<false>(X[2 * w], nm2);
+            p23 = exp2_pair<false>(X[2 * w + 1], nm2);
+          }
+          l2 = f2_add(l2, p01);
+          l2 = f2_add(l2, p23);
+          float2 q01 = f2_mul(p01, c2), q23 = f2_mul(p23, c2);
+          pw[w] = e4m3x4(q01.x, q01.y, q23.x, q23.y);
         }
         tmem_st32(tS + lane_off + T::kPCol, pw);
       } else {
         uint32_t pw[2][32];
 #pragma unroll
         for (int w = 0; w < 64; ++w) {
-          float e0 = ex2_approx(x[2 * w] - m_new), e1 = ex2_approx(x[2 * w + 1] - m_new);
-          lsum += e0 + e1;
-          __nv_bfloat162 pb = __floats2bfloat162_rn(e0, e1);   // .x = e0 in the low half
+          float2 pp = ((w % 8) < kPolyPer8) ? exp2_pair<true>(X[w], nm2) : exp2_pair<false>(X[w], nm2);
+          l2 = f2_add(l2, pp);
+          __nv_bfloat162 pb = __floats2bfloat162_rn(pp.x, pp.y);   // .x in the low half
           pw[w >> 5][w & 31] = *reinterpret_cast<uint32_t*>(&pb);
         }
         tmem_st32(tS + lane_off + T::kPCol, pw[0]);
         tmem_st32(tS + lane_off + T::kPCol + 32, pw[1]);
       }
+      const float lsum = l2.x + l2.y;
       l = l * alpha + lsum;
       m = m_new;
       tmem_wait_st();

@@ -11,6 +11,7 @@
 
 #include "../../include/fqa.h"
 #include "attention.cuh"
+#include "attention_ws.cuh"
 #include "device.cuh"
 #include "quantize.cuh"
 
@@ -23,6 +24,7 @@ constexpr int kMaxDevices = 64;
 struct DeviceCache {
   std::once_flag once;
   uint32_t* status = nullptr;
+  int num_sms = 0;
   cudaError_t err = cudaSuccess;
 };
 DeviceCache g_dev[kMaxDevices];
@@ -41,10 +43,12 @@ static uint32_t* status_ptr(fqa_status* st) {
     return nullptr;
   }
   DeviceCache& c = g_dev[dev];
-  std::call_once(c.once, [&c]() {
+  std::call_once(c.once, [&c, dev]() {
     void* p = nullptr;
     c.err = cudaGetSymbolAddress(&p, g_status_word);
     if (c.err == cudaSuccess) c.status = static_cast<uint32_t*>(p);
+    if (c.err == cudaSuccess)
+      c.err = cudaDeviceGetAttribute(&c.num_sms, cudaDevAttrMultiProcessorCount, dev);
   });
   if (c.err != cudaSuccess || c.status == nullptr) {
     *st = FQA_ERR_CUDA;
@@ -96,6 +100,34 @@ static fqa_status check_shape(int B, int H, int N, int d, int n_mult) {
 
 static fqa_status launch_status() {
   return cudaGetLastError() == cudaSuccess ? FQA_OK : FQA_ERR_CUDA;
+}
+
+static int num_sms() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  return g_dev[dev].num_sms;
+}
+
+// Persistent launch: one CTA per SM (or per work item, if fewer).
+template <bool kFP8>
+static fqa_status launch_attention_ws(const void* q, const void* k, const void* v,
+                                      const AttnParams& prm, cudaStream_t stream) {
+  using T = WsTraits<kFP8>;
+  const uint64_t rows = (uint64_t)prm.B * prm.H * prm.N;
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap(&tq, q, kFP8, rows) || !make_tmap(&tk, k, kFP8, rows) ||
+      !make_tmap(&tv, v, kFP8, rows))
+    return FQA_ERR_CUDA;
+  auto kern = attn_ws_kernel<kFP8>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, T::kSmemBytes) !=
+      cudaSuccess)
+    return FQA_ERR_CUDA;
+  const int items = prm.B * prm.H * ((prm.N + kPairRows - 1) / kPairRows);
+  const int sms = num_sms();
+  if (sms <= 0) return FQA_ERR_CUDA;
+  const int grid = items < sms ? items : sms;
+  kern<<<grid, kWsThreads, T::kSmemBytes, stream>>>(tq, tk, tv, prm);
+  return launch_status();
 }
 
 template <bool kFP8>
@@ -198,7 +230,7 @@ fqa_status fqa_attention_fp8(const void* q8, const void* k8, const void* v8, con
   uint32_t* status = status_ptr(&st);
   if (!status) return st;
   AttnParams prm{B, H, N, softmax_scale, sq, sk, sv, sv_max, out, out_dtype == FQA_OUT_F32, status};
-  return launch_attention<true>(q8, k8, v8, prm, static_cast<cudaStream_t>(cuda_stream));
+  return launch_attention_ws<true>(q8, k8, v8, prm, static_cast<cudaStream_t>(cuda_stream));
 }
 
 fqa_status fqa_attention_bf16(const void* q, const void* k, const void* v, int B, int H, int N,
