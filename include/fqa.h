@@ -85,9 +85,10 @@ FQA_API int fqa_version(void);
 FQA_API const char* fqa_status_string(fqa_status status);
 
 /*
- * Bytes of device workspace fqa_quantize() needs: B*H*(N/64)*d*4 (the
- * per-64-token-block partial sums of the K mean).  Returns 0 for invalid
- * sizes.
+ * Bytes of device workspace fqa_quantize() needs: B*H*(N/64)*d*4 rounded up
+ * to a multiple of 256 (the per-64-token-block partial sums of the K mean),
+ * plus 256 (the launch's grid-barrier and work-queue counters).  Returns 0
+ * for invalid sizes.
  */
 FQA_API size_t fqa_quantize_workspace_bytes(int B, int H, int N, int d);
 
@@ -115,7 +116,10 @@ FQA_API size_t fqa_quantize_workspace_bytes(int B, int H, int N, int d);
  * k_mean       out: FP32 [B,H,d]
  * workspace    scratch of at least fqa_quantize_workspace_bytes(B,H,N,d)
  *              bytes, 16-byte aligned; contents on entry are ignored.
- * Launches three kernels on cuda_stream.
+ * Enqueues on cuda_stream a 16-byte memset of the workspace counters and one
+ * cooperative kernel launch (Q/V codes and K partial sums; K mean and V head
+ * maxima; K codes -- phases separated by bounded grid barriers, 64-token
+ * blocks handed out through work queues).
  */
 FQA_API fqa_status fqa_quantize(const void* q, const void* k, const void* v, int B, int H, int N, int d,
                         void* q8, void* k8, void* v8, float* sq, float* sk, float* sv,
@@ -194,6 +198,15 @@ FQA_API fqa_status fqa_attention_bf16(const void* q, const void* k, const void* 
  * can check the codec exhaustively.  x: FP32 [n], out: uint8 [n] (device).
  */
 FQA_API fqa_status fqa_e4m3_encode(const float* x, uint8_t* out, size_t n, void* cuda_stream);
+
+/*
+ * fqa_debug_wait_timeout -- checks the bounded-wait path (no counterpart on
+ * the pages): launches one thread that waits on an mbarrier nothing arrives
+ * on; after limit_us microseconds (1 .. 2,000,000) the wait gives up, sets the
+ * timeout bit of the device status word and the kernel returns, leaving the
+ * context usable.  The next fqa_debug_status() then returns FQA_ERR_TIMEOUT.
+ */
+FQA_API fqa_status fqa_debug_wait_timeout(uint32_t limit_us, void* cuda_stream);
 
 /*
  * fqa_debug_status -- synchronizes cuda_stream, reads and clears the

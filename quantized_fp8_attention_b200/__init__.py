@@ -138,6 +138,15 @@ def fqa_e4m3_encode(x, out, stream=None) -> int:
     return _load().fqa_e4m3_encode(_ptr(x), _ptr(out), x.numel(), _stream(stream))
 
 
+def fqa_debug_wait_timeout(limit_us: int, stream=None) -> int:
+    """Launch a bounded wait that is bound to give up after limit_us (tests the
+    timeout path; the next fqa_debug_status() reports FQA_ERR_TIMEOUT)."""
+    L = _load()
+    L.fqa_debug_wait_timeout.restype = ctypes.c_int
+    L.fqa_debug_wait_timeout.argtypes = [ctypes.c_uint32, ctypes.c_void_p]
+    return L.fqa_debug_wait_timeout(int(limit_us), _stream(stream))
+
+
 def fqa_debug_status(stream=None):
     """(status, raw flag bits) of the current device's status word; clears it."""
     flags = ctypes.c_uint32(0)

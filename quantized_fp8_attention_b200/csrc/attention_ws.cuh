@@ -315,8 +315,8 @@ __global__ void __launch_bounds__(kWsThreads, 1)
           a0 = a1 = c_log2e;
         }
         // maxima of the raw scores per 64-key half (8 independent chains);
-        // the scales are >= 0, so the tile max of x = fl(S * a) is
-        // max(fl(max S_half0 * a0), fl(max S_half1 * a1)) exactly
+        // the scales are >= 0 and rounding is monotone, so the tile max of
+        // x = S * a (rounded toward zero) is the rounded product of the max
         float cm[8];
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
@@ -328,15 +328,18 @@ __global__ void __launch_bounds__(kWsThreads, 1)
         }
         const float h0 = fmaxf(fmax3(cm[0], cm[1], cm[2]), cm[3]);
         const float h1 = fmaxf(fmax3(cm[4], cm[5], cm[6]), cm[7]);
+        // x = S * a rounded once, toward zero: a rounding ptxas cannot fuse
+        // into the next step, fma(x, 1, -m), so the row maximum gets p = 1
+        // exactly and x - m is exact near the maximum
         float2 X[64];
 #pragma unroll
         for (int e = 0; e < 64; ++e) {
           const float a = (e < 32) ? a0 : a1;
-          X[e] = f2_mul(make_float2(__uint_as_float(sr[e >> 4][(2 * e) & 31]),
-                                    __uint_as_float(sr[e >> 4][(2 * e + 1) & 31])),
-                        make_float2(a, a));
+          X[e] = f2_mul_rz(make_float2(__uint_as_float(sr[e >> 4][(2 * e) & 31]),
+                                       __uint_as_float(sr[e >> 4][(2 * e + 1) & 31])),
+                           make_float2(a, a));
         }
-        const float m_new = fmaxf(m, fmaxf(h0 * a0, h1 * a1));
+        const float m_new = fmaxf(m, fmaxf(__fmul_rz(h0, a0), __fmul_rz(h1, a1)));
         const float alpha = ex2_approx(m - m_new);
         const float2 nm2 = make_float2(-m_new, -m_new);
         // Ping-pong: the two warpgroups take turns for the exponential loop

@@ -69,21 +69,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // (after flagging the CTA-wide abort word and the device status word) if the
 // phase did not complete within kWaitLimitNs, or if another warp of the CTA
 // already aborted.  Never traps.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          uint32_t* status) {
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity,
+                                                volatile int* abort_flag, uint32_t* status,
+                                                uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 63u) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         *abort_flag = 1;
         atomicOr(status, kStatusTimeout);
         return false;
       }
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          uint32_t* status) {
+  return mbar_wait_limit(bar, parity, abort_flag, status, kWaitLimitNs);
 }
 
 // ------------------------------------------------------------------ TMA
@@ -101,6 +106,36 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(smem_dst)),
       "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(x), "r"(y)
       : "memory");
+}
+
+// L2 eviction policies for cache-hinted accesses.
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// 1-D bulk copy global -> shared (addresses 16-byte aligned, size a
+// multiple of 16), completing on `bar`, with an L2 eviction policy.
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes,
+                                          uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], "
+      "%2, [%3], %4;" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+// 8-byte global store with an L2 eviction policy (no L1 allocation).
+__device__ __forceinline__ void st_global_v2_hint(void* gdst, uint32_t a, uint32_t b, uint64_t policy) {
+  asm volatile("st.global.L1::no_allocate.L2::cache_hint.v2.b32 [%0], {%1, %2}, %3;" ::"l"(gdst),
+               "r"(a), "r"(b), "l"(policy)
+               : "memory");
 }
 
 // -------------------------------------------------------------- tcgen05
@@ -260,6 +295,15 @@ __device__ __forceinline__ uint32_t e4m3x4(float v0, float v1, float v2, float v
 __device__ __forceinline__ float2 f2_mul(float2 a, float2 b) {
   float2 c;
   asm("mul.rn.f32x2 %0, %1, %2;"
+      : "=l"(reinterpret_cast<uint64_t&>(c))
+      : "l"(reinterpret_cast<uint64_t&>(a)), "l"(reinterpret_cast<uint64_t&>(b)));
+  return c;
+}
+// Round-toward-zero product: the explicit non-default rounding keeps ptxas
+// from contracting it with a following add/fma into one fused operation.
+__device__ __forceinline__ float2 f2_mul_rz(float2 a, float2 b) {
+  float2 c;
+  asm("mul.rz.f32x2 %0, %1, %2;"
       : "=l"(reinterpret_cast<uint64_t&>(c))
       : "l"(reinterpret_cast<uint64_t&>(a)), "l"(reinterpret_cast<uint64_t&>(b)));
   return c;

@@ -130,24 +130,6 @@ static fqa_status launch_attention_ws(const void* q, const void* k, const void* 
   return launch_status();
 }
 
-template <bool kFP8>
-static fqa_status launch_attention(const void* q, const void* k, const void* v, const AttnParams& prm,
-                                   cudaStream_t stream) {
-  using T = AttnTraits<kFP8>;
-  const uint64_t rows = (uint64_t)prm.B * prm.H * prm.N;
-  CUtensorMap tq, tk, tv;
-  if (!make_tmap(&tq, q, kFP8, rows) || !make_tmap(&tk, k, kFP8, rows) ||
-      !make_tmap(&tv, v, kFP8, rows))
-    return FQA_ERR_CUDA;
-  auto kern = attn_fwd_kernel<kFP8>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, T::kSmemBytes) !=
-      cudaSuccess)
-    return FQA_ERR_CUDA;
-  dim3 grid(prm.N / kBlockM, prm.H, prm.B);
-  kern<<<grid, kAttnThreads, T::kSmemBytes, stream>>>(tq, tk, tv, prm);
-  return launch_status();
-}
-
 }  // namespace fqa
 
 using namespace fqa;
@@ -168,9 +150,15 @@ const char* fqa_status_string(fqa_status s) {
   return "FQA_UNKNOWN_STATUS";
 }
 
+// Workspace: the K-mean partial sums [B,H,N/64,128] FP32, then (256-byte
+// aligned) the grid-barrier counter of the fused quantize launch.
+static size_t partial_bytes(int B, int H, int N, int d) {
+  return (size_t)B * H * (N / kQBlock) * d * sizeof(float);
+}
+
 size_t fqa_quantize_workspace_bytes(int B, int H, int N, int d) {
   if (check_shape(B, H, N, d, kQBlock) != FQA_OK) return 0;
-  return (size_t)B * H * (N / kQBlock) * d * sizeof(float);
+  return ((partial_bytes(B, H, N, d) + 255) & ~size_t(255)) + 256;
 }
 
 fqa_status fqa_quantize(const void* q, const void* k, const void* v, int B, int H, int N, int d,
@@ -189,15 +177,39 @@ fqa_status fqa_quantize(const void* q, const void* k, const void* v, int B, int 
   const void* a4[] = {sq, sk, sv, sv_max, k_mean};
   for (const void* p : a4)
     if (!aligned(p, 4)) return FQA_ERR_MISALIGNED;
+  uint32_t* status = status_ptr(&st);
+  if (!status) return st;
   cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
   float* partial = static_cast<float*>(workspace);
-  dim3 grid(N / kQBlock, H, B);
-  kmean_partial_kernel<<<grid, 128, 0, s>>>(static_cast<const __nv_bfloat16*>(k), partial, H, N);
-  kmean_reduce_kernel<<<B * H, 128, 0, s>>>(partial, k_mean, sv_max, N);
-  quantize_qkv_kernel<<<grid, 256, 0, s>>>(
-      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-      static_cast<const __nv_bfloat16*>(v), k_mean, static_cast<uint8_t*>(q8),
-      static_cast<uint8_t*>(k8), static_cast<uint8_t*>(v8), sq, sk, sv, sv_max, H, N);
+  unsigned int* ctr = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(workspace) +
+                                                      ((partial_bytes(B, H, N, d) + 255) & ~size_t(255)));
+  const int nunits = B * H * (N / kQBlock);
+  if (cudaFuncSetAttribute(quantize_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kQuantSmem) != cudaSuccess)
+    return FQA_ERR_CUDA;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quantize_fused_kernel, kQuantThreads,
+                                                    kQuantSmem) != cudaSuccess ||
+      per_sm < 1)
+    return FQA_ERR_CUDA;
+  int grid = per_sm * num_sms();
+  if (grid > nunits) grid = nunits;
+  static_assert(kNumCtr * sizeof(unsigned int) <= 256, "counters fit the reserved 256 bytes");
+  if (cudaMemsetAsync(ctr, 0, kNumCtr * sizeof(unsigned int), s) != cudaSuccess) return FQA_ERR_CUDA;
+  const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(q);
+  const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(k);
+  const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(v);
+  uint8_t* q8b = static_cast<uint8_t*>(q8);
+  uint8_t* k8b = static_cast<uint8_t*>(k8);
+  uint8_t* v8b = static_cast<uint8_t*>(v8);
+  void* args[] = {(void*)&qb, (void*)&kb, (void*)&vb, (void*)&q8b, (void*)&k8b, (void*)&v8b,
+                  (void*)&sq, (void*)&sk, (void*)&sv, (void*)&sv_max, (void*)&k_mean,
+                  (void*)&partial, (void*)&ctr, (void*)&B, (void*)&H, (void*)&N, (void*)&status};
+  // cooperative: every CTA is resident, so the grid barriers cannot wait on
+  // a CTA that never starts
+  if (cudaLaunchCooperativeKernel((const void*)quantize_fused_kernel, dim3(grid), dim3(kQuantThreads),
+                                  args, kQuantSmem, s) != cudaSuccess)
+    return FQA_ERR_CUDA;
   return launch_status();
 }
 
@@ -247,7 +259,7 @@ fqa_status fqa_attention_bf16(const void* q, const void* k, const void* v, int B
   if (!status) return st;
   AttnParams prm{B, H, N, softmax_scale, nullptr, nullptr, nullptr, nullptr, out,
                  out_dtype == FQA_OUT_F32, status};
-  return launch_attention<false>(q, k, v, prm, static_cast<cudaStream_t>(cuda_stream));
+  return launch_attention_ws<false>(q, k, v, prm, static_cast<cudaStream_t>(cuda_stream));
 }
 
 fqa_status fqa_e4m3_encode(const float* x, uint8_t* out, size_t n, void* cuda_stream) {
@@ -255,6 +267,16 @@ fqa_status fqa_e4m3_encode(const float* x, uint8_t* out, size_t n, void* cuda_st
   if (n == 0) return FQA_OK;
   if (!aligned(x, 4)) return FQA_ERR_MISALIGNED;
   e4m3_encode_kernel<<<148 * 8, 256, 0, static_cast<cudaStream_t>(cuda_stream)>>>(x, out, n);
+  return launch_status();
+}
+
+fqa_status fqa_debug_wait_timeout(uint32_t limit_us, void* cuda_stream) {
+  if (limit_us == 0 || limit_us > 2000000u) return FQA_ERR_INVALID_ARG;
+  fqa_status st = FQA_OK;
+  uint32_t* status = status_ptr(&st);
+  if (!status) return st;
+  wait_timeout_kernel<<<1, 1, 0, static_cast<cudaStream_t>(cuda_stream)>>>(
+      status, (uint64_t)limit_us * 1000ull);
   return launch_status();
 }
 

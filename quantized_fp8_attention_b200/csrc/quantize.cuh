@@ -14,139 +14,332 @@
 //   s      = amax / 448, inv = 448 / amax (RN divisions; 0 and 0 if amax = 0);
 //   code   = E4M3_RNE_satfinite(fl32(x * inv));
 //   sv_max = max over the head's V block scales.
-// All three kernels read BF16 [B,H,N,128] and write codes in the same layout.
+// Inputs are BF16 [B,H,N,128]; codes are written in the same layout.
 #pragma once
 
 #include "device.cuh"
 
 namespace fqa {
 
-// Level 1 of the K mean: partial[b,h,j,c] = sequential sum of the block's 64
-// tokens of channel c.  grid (N/64, H, B), 128 threads (one per channel).
-__global__ void __launch_bounds__(128) kmean_partial_kernel(const __nv_bfloat16* __restrict__ k,
-                                                            float* __restrict__ partial, int H,
-                                                            int N) {
-  const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z, c = threadIdx.x;
-  const size_t head = (size_t)b * H + h;
-  const __nv_bfloat16* src = k + (head * N + (size_t)j * kQBlock) * kHeadDim + c;
-  float v[kQBlock];
-#pragma unroll
-  for (int n = 0; n < kQBlock; ++n) v[n] = __bfloat162float(src[(size_t)n * kHeadDim]);
-  float p = 0.0f;
-#pragma unroll
-  for (int n = 0; n < kQBlock; ++n) p = __fadd_rn(p, v[n]);
-  partial[(head * (N / kQBlock) + j) * kHeadDim + c] = p;
-}
+// ---------------------------------------------------------------------------
+// Fused quantizer: one cooperative persistent launch in three phases separated
+// by grid barriers (the K codes need the K mean, which needs all of K):
+//   1a  Q and V units -> codes and scales
+//   1b  K units -> per-unit partial sums (per channel, 64 tokens in order);
+//       K read last and marked evict-last in L2 for phase 3
+//   2   per (b, h): k_mean from the partials in block order; sv_max = max of
+//       the V unit scales (no atomics)
+//   3   K units -> smoothed codes and scales, newest units of 1b first
+// Unit u = (b*H + h)*(N/64) + j is one 64-token block of one head: 16 KB of
+// contiguous BF16 per tensor.  Units are handed out through work queues
+// (counters the launch zeroes), so the SMs that stream faster take more.
+// All loads are 1-D bulk copies into a shared-memory ring of kRingBytes, cut
+// into as many slots as the phase's unit size allows, so each SM keeps several
+// units in flight.  Thread t handles the 16-byte chunks t, t+T, t+2T, ... of
+// a unit (T threads, 8 channels a chunk).  Every wait is bounded.
 
-// Level 2: mu = (sequential sum of the partials over blocks) / N; also
-// clears sv_max for the quantize kernel's atomic maximum.
-// grid (B*H), 128 threads.
-__global__ void __launch_bounds__(128) kmean_reduce_kernel(const float* __restrict__ partial,
-                                                           float* __restrict__ k_mean,
-                                                           float* __restrict__ sv_max, int N) {
-  const size_t head = blockIdx.x;
-  const int c = threadIdx.x, nblk = N / kQBlock;
-  const float* src = partial + head * nblk * kHeadDim + c;
-  float t = 0.0f;
-  for (int j = 0; j < nblk; ++j) t = __fadd_rn(t, src[(size_t)j * kHeadDim]);
-  k_mean[head * kHeadDim + c] = __fdiv_rn(t, (float)N);
-  if (c == 0) sv_max[head] = 0.0f;
-}
+#ifndef FQA_QUANT_THREADS
+#define FQA_QUANT_THREADS 256
+#endif
+#ifndef FQA_QUANT_RING_KB
+#define FQA_QUANT_RING_KB 64
+#endif
+constexpr int kQuantThreads = FQA_QUANT_THREADS;
+constexpr int kQuantWarps = kQuantThreads / 32;
+constexpr int kBlockBytes = kQBlock * kHeadDim * 2;            // 16 KB of BF16
+constexpr int kChunks = kBlockBytes / 16 / kQuantThreads;       // 16-byte chunks per thread
+constexpr int kVals = 8 * kChunks;
+constexpr int kRingBytes = FQA_QUANT_RING_KB * 1024;
+constexpr int kMaxSlots = kRingBytes / kBlockBytes;
+constexpr int kQuantSmem = kRingBytes + 128;
+constexpr int kPartialRowsPerSlot = kBlockBytes / (kHeadDim * 4);   // 32 partial rows per 16 KB
+// CTAs the shared memory admits per SM (the register cap follows from it)
+constexpr int kQuantMinCtas = (200 * 1024) / (kQuantSmem + 2048) < 1 ? 1 : (200 * 1024) / (kQuantSmem + 2048);
+static_assert(kMaxSlots >= 4 && kMaxSlots <= 32, "ring size");
+static_assert(kQuantThreads >= 2 * kHeadDim, "k_mean and sv_max threads");
+static_assert((kQuantThreads * 8) % kHeadDim == 0, "chunk c of thread t starts at channel 8t mod 128");
 
-__device__ __forceinline__ float block_max_256(float v, float* red, int slot) {
-  // max over the 256 threads of the CTA; red holds 8 floats for this slot
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  if ((threadIdx.x & 31) == 0) red[slot * 8 + (threadIdx.x >> 5)] = v;
-  return v;
-}
+// Counters the launch zeroes (in the workspace, after the partial sums).
+constexpr int kCtrBarrier = 0;     // grid barrier arrivals
+constexpr int kCtrQV = 1;          // next unit of phase 1a
+constexpr int kCtrK = 2;           // next unit of phase 1b
+constexpr int kCtrK3 = 3;          // next unit of phase 3 (counted from the end)
+constexpr int kNumCtr = 4;
 
-// One CTA quantizes one 64-token block of Q, K and V for one (b, h).
-// Thread t owns token row t/4 and channels [32*(t%4), 32*(t%4)+32).
-// grid (N/64, H, B), 256 threads.
-__global__ void __launch_bounds__(256) quantize_qkv_kernel(
-    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-    const __nv_bfloat16* __restrict__ v, const float* __restrict__ k_mean,
-    uint8_t* __restrict__ q8, uint8_t* __restrict__ k8, uint8_t* __restrict__ v8,
-    float* __restrict__ sq, float* __restrict__ sk, float* __restrict__ sv,
-    float* __restrict__ sv_max, int H, int N) {
-  __shared__ float red[3 * 8];
-  __shared__ float mu[kHeadDim];
-  const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int t = threadIdx.x, row = t >> 2, c0 = (t & 3) * 32;
-  const size_t head = (size_t)b * H + h;
-  const size_t elem0 = (head * N + (size_t)j * kQBlock + row) * kHeadDim + c0;
-
-  // issue all global loads first: 3 tensors x 64 bytes per thread
-  uint4 raw[3][4];
-  const uint4* srcq = reinterpret_cast<const uint4*>(q + elem0);
-  const uint4* srck = reinterpret_cast<const uint4*>(k + elem0);
-  const uint4* srcv = reinterpret_cast<const uint4*>(v + elem0);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    raw[0][i] = __ldg(srcq + i);
-    raw[1][i] = __ldg(srck + i);
-    raw[2][i] = __ldg(srcv + i);
-  }
-  if (t < kHeadDim) mu[t] = k_mean[head * kHeadDim + t];
+// Grid barrier number `round` (1, 2, ...): arrive, then wait until every CTA
+// of the grid has arrived `round` times.  Gives up after kWaitLimitNs.
+__device__ __forceinline__ bool grid_barrier(unsigned int* ctr, unsigned int round, uint32_t* status,
+                                             volatile int* failed) {
   __syncthreads();
-
-  float x[3][32];
-#pragma unroll
-  for (int s = 0; s < 3; ++s) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw[s][i]);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        float2 f = __bfloat1622float2(h2[e]);
-        x[s][i * 8 + 2 * e] = f.x;
-        x[s][i * 8 + 2 * e + 1] = f.y;
+  if (threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(ctr, 1u);
+    const unsigned int target = round * gridDim.x;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+      unsigned int v = *reinterpret_cast<volatile unsigned int*>(ctr);
+      if ((int)(v - target) >= 0) break;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        atomicOr(status, kStatusTimeout);
+        *failed = 1;
+        break;
       }
+      __nanosleep(64);
     }
-  }
-#pragma unroll
-  for (int i = 0; i < 32; ++i) x[1][i] = __fsub_rn(x[1][i], mu[c0 + i]);
-
-  float amax[3];
-#pragma unroll
-  for (int s = 0; s < 3; ++s) {
-    float m = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(x[s][i]));
-    block_max_256(m, red, s);
+    __threadfence();
+    // what other CTAs wrote before the barrier is read next by bulk copies
+    asm volatile("fence.proxy.async.global;" ::: "memory");
   }
   __syncthreads();
-#pragma unroll
-  for (int s = 0; s < 3; ++s) {
-    float m = red[s * 8];
-#pragma unroll
-    for (int w = 1; w < 8; ++w) m = fmaxf(m, red[s * 8 + w]);
-    amax[s] = m;
-  }
+  return *failed == 0;
+}
 
-  uint8_t* dst[3] = {q8, k8, v8};
-  float* scl[3] = {sq, sk, sv};
+// The values of this thread's chunks of a staged BF16 unit.
+__device__ __forceinline__ void chunks_to_f32(const uint8_t* blk, float (&x)[kVals]) {
 #pragma unroll
-  for (int s = 0; s < 3; ++s) {
-    const float a = amax[s];
-    const float scale = a > 0.0f ? __fdiv_rn(a, 448.0f) : 0.0f;
-    const float inv = a > 0.0f ? __fdiv_rn(448.0f, a) : 0.0f;
-    uint32_t w[8];
+  for (int i = 0; i < kChunks; ++i) {
+    const uint4 raw = *reinterpret_cast<const uint4*>(blk + 16 * (threadIdx.x + kQuantThreads * i));
+    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      uint32_t lo = e4m3x2(__fmul_rn(x[s][4 * i], inv), __fmul_rn(x[s][4 * i + 1], inv));
-      uint32_t hi = e4m3x2(__fmul_rn(x[s][4 * i + 2], inv), __fmul_rn(x[s][4 * i + 3], inv));
-      w[i] = lo | (hi << 16);
-    }
-    uint4* o = reinterpret_cast<uint4*>(dst[s] + elem0);
-    o[0] = make_uint4(w[0], w[1], w[2], w[3]);
-    o[1] = make_uint4(w[4], w[5], w[6], w[7]);
-    if (t == 0) {
-      scl[s][head * (N / kQBlock) + j] = scale;
-      if (s == 2) atomicMax(reinterpret_cast<unsigned int*>(sv_max + head), __float_as_uint(scale));
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __bfloat1622float2(h2[e]);
+      x[i * 8 + 2 * e] = f.x;
+      x[i * 8 + 2 * e + 1] = f.y;
     }
   }
+}
+
+// Block absmax over the CTA (red: one float per warp for this slot), scale,
+// and the codes of this thread's chunks (8 bytes per chunk, chunk c at byte 8c).
+__device__ __forceinline__ float quantize_chunks(float (&x)[kVals], float* red, uint8_t* dst, int slot,
+                                                 uint64_t policy) {
+  const int t = threadIdx.x;
+  float m = 0.0f;
+#pragma unroll
+  for (int i = 0; i < kVals; ++i) m = fmaxf(m, fabsf(x[i]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((t & 31) == 0) red[slot * kQuantWarps + (t >> 5)] = m;
+  __syncthreads();
+  float a = red[slot * kQuantWarps];
+#pragma unroll
+  for (int w = 1; w < kQuantWarps; ++w) a = fmaxf(a, red[slot * kQuantWarps + w]);
+  const float scale = a > 0.0f ? __fdiv_rn(a, 448.0f) : 0.0f;
+  const float inv = a > 0.0f ? __fdiv_rn(448.0f, a) : 0.0f;
+#pragma unroll
+  for (int i = 0; i < kChunks; ++i) {
+    uint32_t lo = e4m3x2(__fmul_rn(x[8 * i], inv), __fmul_rn(x[8 * i + 1], inv));
+    uint32_t hi = e4m3x2(__fmul_rn(x[8 * i + 2], inv), __fmul_rn(x[8 * i + 3], inv));
+    uint32_t lo2 = e4m3x2(__fmul_rn(x[8 * i + 4], inv), __fmul_rn(x[8 * i + 5], inv));
+    uint32_t hi2 = e4m3x2(__fmul_rn(x[8 * i + 6], inv), __fmul_rn(x[8 * i + 7], inv));
+    st_global_v2_hint(dst + 8 * (t + kQuantThreads * i), lo | (hi << 16), lo2 | (hi2 << 16), policy);
+  }
+  return scale;
+}
+
+__global__ void __launch_bounds__(kQuantThreads, kQuantMinCtas) quantize_fused_kernel(
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+    const __nv_bfloat16* __restrict__ v, uint8_t* __restrict__ q8, uint8_t* __restrict__ k8,
+    uint8_t* __restrict__ v8, float* __restrict__ sq, float* __restrict__ sk,
+    float* __restrict__ sv, float* __restrict__ sv_max, float* __restrict__ k_mean,
+    float* __restrict__ partial, unsigned int* __restrict__ ctr, int B, int H, int N,
+    uint32_t* status) {
+  extern __shared__ uint8_t qsmem_raw[];
+  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(qsmem_raw) + 127) & ~uintptr_t(127));
+  __shared__ uint64_t full[kMaxSlots];
+  __shared__ int slot_unit[kMaxSlots];
+  __shared__ float red[2 * kQuantWarps];
+  __shared__ float mu[kHeadDim];
+  __shared__ int failed, abort_flag;
+  const int t = threadIdx.x;
+  const int nblk = N / kQBlock;
+  const int nunits = B * H * nblk;
+  const int G = gridDim.x;
+  if (t == 0) {
+    failed = 0;
+    abort_flag = 0;
+    for (int s = 0; s < kMaxSlots; ++s) mbar_init(&full[s], 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  const uint64_t pol_first = l2_policy_evict_first();
+  const uint64_t pol_last = l2_policy_evict_last();
+  uint32_t phase_bits = 0;                         // parity of each ring barrier
+
+  // One pipelined pass with slots of slot_bytes.  next() (thread 0) yields
+  // the next unit index, or -1 when there is none and from then on;
+  // issue(u, dst, bar) starts unit u's bulk copies (it arms bar itself);
+  // body(u, slot memory) runs on all threads, in the order next() gave the
+  // units.  Every started copy is waited for before the pass returns, unless
+  // a wait timed out (returns false).
+  auto run = [&](int slot_bytes, auto next, auto issue, auto body) -> bool {
+    const int nslots = kRingBytes / slot_bytes;
+    if (t == 0)
+      for (int s = 0; s < nslots - 1; ++s) {
+        const int u = next();
+        slot_unit[s] = u;
+        if (u >= 0) issue(u, ring + s * slot_bytes, &full[s]);
+      }
+    __syncthreads();
+    for (int s = 0;; s = (s + 1 == nslots) ? 0 : s + 1) {
+      const int u = slot_unit[s];
+      if (u < 0) break;                            // CTA-uniform
+      if (t == 0) {
+        // the slot before s was released by the barrier that ended its unit
+        const int s2 = (s == 0) ? nslots - 1 : s - 1;
+        const int u2 = next();
+        slot_unit[s2] = u2;
+        if (u2 >= 0) issue(u2, ring + s2 * slot_bytes, &full[s2]);
+      }
+      const bool ok = mbar_wait(&full[s], (phase_bits >> s) & 1u, &abort_flag, status);
+      phase_bits ^= 1u << s;
+      if (!__syncthreads_and(ok)) return false;
+      body(u, ring + s * slot_bytes);
+      __syncthreads();                             // slot s, slot_unit and red free again
+    }
+    return true;
+  };
+  // a shared work queue over all units: ctr[c] counts the units handed out
+  auto queue = [&](int c, bool reverse) {
+    bool drained = false;
+    return [=]() mutable -> int {
+      if (drained) return -1;
+      const unsigned int i = atomicAdd(&ctr[c], 1u);
+      if (i >= (unsigned int)nunits) {
+        drained = true;
+        return -1;
+      }
+      return reverse ? nunits - 1 - (int)i : (int)i;
+    };
+  };
+  auto blk_ptr = [&](const __nv_bfloat16* base, int u) {
+    return base + (size_t)u * kQBlock * kHeadDim;
+  };
+
+  // ---- phase 1a: Q and V (streamed once: evict-first)
+  bool ok = run(2 * kBlockBytes, queue(kCtrQV, false),
+      [&](int u, uint8_t* dst, uint64_t* bar) {
+        mbar_arrive_expect_tx(bar, 2 * kBlockBytes);
+        bulk_load(dst, blk_ptr(q, u), kBlockBytes, bar, pol_first);
+        bulk_load(dst + kBlockBytes, blk_ptr(v, u), kBlockBytes, bar, pol_first);
+      },
+      [&](int u, const uint8_t* blk) {
+        const size_t off = (size_t)u * kQBlock * kHeadDim;
+        float x[kVals];
+        chunks_to_f32(blk, x);
+        const float s_q = quantize_chunks(x, red, q8 + off, 0, pol_first);
+        chunks_to_f32(blk + kBlockBytes, x);
+        const float s_v = quantize_chunks(x, red, v8 + off, 1, pol_first);
+        if (t == 0) {
+          sq[u] = s_q;
+          sv[u] = s_v;
+        }
+      });
+  // ---- phase 1b: K partial sums (one thread per channel adds the unit's 64
+  // tokens in order); K stays in L2 for phase 3
+  if (ok)
+    ok = run(kBlockBytes, queue(kCtrK, false),
+        [&](int u, uint8_t* dst, uint64_t* bar) {
+          mbar_arrive_expect_tx(bar, kBlockBytes);
+          bulk_load(dst, blk_ptr(k, u), kBlockBytes, bar, pol_last);
+        },
+        [&](int u, const uint8_t* blk) {
+          if (t < kHeadDim) {
+            const __nv_bfloat16* kb = reinterpret_cast<const __nv_bfloat16*>(blk);
+            float acc = 0.0f;
+#pragma unroll 16
+            for (int n = 0; n < kQBlock; ++n) acc = __fadd_rn(acc, __bfloat162float(kb[n * kHeadDim + t]));
+            partial[(size_t)u * kHeadDim + t] = acc;
+          }
+        });
+  if (!ok) failed = 1;
+  if (!grid_barrier(&ctr[kCtrBarrier], 1, status, &failed)) return;
+
+  // ---- phase 2: per (b, h), k_mean (threads 0..127: one channel each, the
+  // partials staged 32 rows a slot and added in block order) and sv_max
+  // (threads 128..255: a max over the V unit scales, any order; the scales
+  // come from other SMs, so the loads bypass L1)
+  for (int hd = blockIdx.x; hd < B * H; hd += G) {
+    if (t >= kHeadDim && t < 2 * kHeadDim) {
+      float m = 0.0f;
+      for (int j = t - kHeadDim; j < nblk; j += kHeadDim) m = fmaxf(m, __ldcg(sv + (size_t)hd * nblk + j));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      if ((t & 31) == 0) red[kQuantWarps + ((t - kHeadDim) >> 5)] = m;
+    }
+    const float* src = partial + (size_t)hd * nblk * kHeadDim;
+    const int nchunk = (nblk + kPartialRowsPerSlot - 1) / kPartialRowsPerSlot;
+    int next_chunk = 0;
+    float acc = 0.0f;
+    ok = run(kBlockBytes, [&]() -> int { return next_chunk < nchunk ? next_chunk++ : -1; },
+        [&](int i, uint8_t* dst, uint64_t* bar) {
+          const int rows = min(kPartialRowsPerSlot, nblk - i * kPartialRowsPerSlot);
+          mbar_arrive_expect_tx(bar, rows * kHeadDim * 4);
+          bulk_load(dst, src + (size_t)i * kPartialRowsPerSlot * kHeadDim, rows * kHeadDim * 4, bar,
+                    pol_first);
+        },
+        [&](int i, const uint8_t* blk) {
+          if (t < kHeadDim) {
+            const float* pr = reinterpret_cast<const float*>(blk);
+            const int rows = min(kPartialRowsPerSlot, nblk - i * kPartialRowsPerSlot);
+#pragma unroll 8
+            for (int r = 0; r < rows; ++r) acc = __fadd_rn(acc, pr[r * kHeadDim + t]);
+          }
+        });
+    if (!ok) {
+      failed = 1;
+      break;
+    }
+    if (t < kHeadDim) k_mean[(size_t)hd * kHeadDim + t] = __fdiv_rn(acc, (float)N);
+    if (t == kHeadDim) {
+      float m = red[kQuantWarps];
+#pragma unroll
+      for (int w = 1; w < kHeadDim / 32; ++w) m = fmaxf(m, red[kQuantWarps + w]);
+      sv_max[hd] = m;
+    }
+    __syncthreads();                               // red reused by the next head
+  }
+  if (!grid_barrier(&ctr[kCtrBarrier], 2, status, &failed)) return;
+
+  // ---- phase 3: K codes, newest units of phase 1b first
+  int last_head = -1;
+  float mr[8];                                     // k_mean of this thread's 8 channels
+  run(kBlockBytes, queue(kCtrK3, true),
+      [&](int u, uint8_t* dst, uint64_t* bar) {
+        mbar_arrive_expect_tx(bar, kBlockBytes);
+        bulk_load(dst, blk_ptr(k, u), kBlockBytes, bar, pol_first);
+      },
+      [&](int u, const uint8_t* blk) {
+        const int head = u / nblk;
+        if (head != last_head) {                   // CTA-uniform
+          if (t < kHeadDim) mu[t] = __ldcg(k_mean + (size_t)head * kHeadDim + t);
+          __syncthreads();
+          // every chunk of this thread starts at channel 8t mod 128
+#pragma unroll
+          for (int e = 0; e < 8; ++e) mr[e] = mu[((8 * t) & (kHeadDim - 1)) + e];
+          last_head = head;
+        }
+        float x[kVals];
+        chunks_to_f32(blk, x);
+#pragma unroll
+        for (int i4 = 0; i4 < kChunks; ++i4)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[8 * i4 + e] = __fsub_rn(x[8 * i4 + e], mr[e]);
+        const float s_k = quantize_chunks(x, red, k8 + (size_t)u * kQBlock * kHeadDim, 0, pol_first);
+        if (t == 0) sk[u] = s_k;
+      });
+}
+
+// Exercises the bounded-wait path: one thread waits on an mbarrier that no
+// one arrives on; after limit_ns the wait gives up, sets the timeout bit of
+// the status word and the kernel returns normally.
+__global__ void wait_timeout_kernel(uint32_t* status, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  mbar_init(&bar, 1);
+  abort_flag = 0;
+  mbar_fence_init();
+  mbar_wait_limit(&bar, 0, &abort_flag, status, limit_ns);
 }
 
 // Standalone conversion kernel: every binary32 input -> its E4M3 code via the

@@ -46,8 +46,11 @@ def test_status_strings_and_version(L):
 
 def test_workspace_bytes(L):
     import quantized_fp8_attention_b200 as fqa
-    assert fqa.fqa_quantize_workspace_bytes(1, 24, 8704) == 24 * 136 * 128 * 4
-    assert fqa.fqa_quantize_workspace_bytes(2, 24, 16896) == 2 * 24 * 264 * 128 * 4
+    r256 = lambda x: (x + 255) // 256 * 256
+    ws = lambda B, H, N: r256(B * H * (N // 64) * 128 * 4) + 256
+    assert fqa.fqa_quantize_workspace_bytes(1, 24, 8704) == ws(1, 24, 8704) == 1671168 + 256
+    assert fqa.fqa_quantize_workspace_bytes(2, 24, 16896) == ws(2, 24, 16896)
+    assert fqa.fqa_quantize_workspace_bytes(1, 65535, 64) == ws(1, 65535, 64)
     assert fqa.fqa_quantize_workspace_bytes(1, 1, 100) == 0       # N % 64 != 0
     assert fqa.fqa_quantize_workspace_bytes(1, 1, 128, 64) == 0   # d != 128
 
@@ -102,3 +105,6 @@ def test_attention_validation(L):
     assert bf(scale=-1.0) == 1
     assert bf(q=_p(0x10002)) == 3
     assert L.fqa_e4m3_encode(None, ok, 4, None) == 1
+    L.fqa_debug_wait_timeout.argtypes = [ctypes.c_uint32, P]
+    assert L.fqa_debug_wait_timeout(0, None) == 1
+    assert L.fqa_debug_wait_timeout(3000000, None) == 1

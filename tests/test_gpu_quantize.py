@@ -104,3 +104,20 @@ def test_quantize_rejects_bad_arguments():
     raw = torch.zeros(128 * 128 + 8, dtype=torch.bfloat16, device="cuda")
     mis = raw[1:1 + 128 * 128].view(1, 1, 128, 128)                        # 2-byte offset
     assert fqa.fqa_quantize(mis, t, t, *qz, ws) == fqa.FQA_ERR_MISALIGNED
+
+
+def test_bounded_wait_times_out_and_context_survives():
+    """A wait on a barrier nothing arrives on gives up after its limit, sets the
+    timeout bit, and leaves the context usable (no trap, no hang)."""
+    fqa = _fqa()
+    assert fqa.fqa_debug_status()[0] == fqa.FQA_OK
+    assert fqa.fqa_debug_wait_timeout(20000) == fqa.FQA_OK      # 20 ms
+    st, flags = fqa.fqa_debug_status()
+    assert st == fqa.FQA_ERR_TIMEOUT and flags & 1
+    assert fqa.fqa_debug_status()[0] == fqa.FQA_OK              # cleared by the read
+    # the context still runs kernels correctly
+    g = U.host_inputs(0)
+    q, k, v = (U.to_device(g[t]) for t in "qkv")
+    got = U.to_oracle_quant(fqa.quantize(q, k, v))
+    ref = U.oracle_quant(0)
+    assert np.array_equal(got["q8"], ref["q8"])
