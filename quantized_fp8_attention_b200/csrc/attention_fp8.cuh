@@ -1,0 +1,485 @@
+// attention_fp8.cuh -- persistent FP8 attention forward on tcgen05, with P
+// staged through shared memory so that a Q tile's next S = Q K^T overlaps
+// its current softmax, and each score row split between two threads.
+//
+// Arithmetic: the per-row rule of attention.cuh (FP8 scaled dot-product
+// attention with Q, K, V as E4M3 codes and per-64-token block scales, "NVIDIA
+// RTX AI optimiert FLUX.1 fuer Bilddaten mit niedriger Genauigkeit", SDPA
+// quantization paragraph).
+//
+// Organisation (one CTA per SM, persistent over work items):
+//   work item   = (b, h, pair of 128-row Q tiles); items taken round-robin
+//   warps 0-15  softmax: warpgroup 2t+hf handles Q tile t, keys [64hf, 64hf+64)
+//               of every KV tile (thread = row = TMEM lane)
+//   warp 16     TMA producer: Q0, Q1 per item; K tiles through a ring
+//   warp 17     TMEM allocator; tcgen05.mma issuer of Q tile 0
+//   warp 18     TMA producer: V tiles through a ring
+//   warp 19     tcgen05.mma issuer of Q tile 1
+// TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).
+// Shared memory: Q0, Q1; kStages K and V tiles; P_t in two buffers per Q
+// tile (128 rows x 128 keys E4M3, the K-major 128-byte-swizzled layout the
+// MMA reads as its A operand); the halves' row sums at the end of an item.
+//
+// Per KV tile g of the CTA's work, each softmax thread (row r, half hf):
+//   wait S_t(g) -> tcgen05.ld the other half's 64 scores, then its own 64
+//   -> row max over all 128 keys (both halves compute the same value), x,
+//   alpha -> exponentials of its 64 keys (the second 32 scores read again
+//   halfway, after which barSfree lets S_t(g+1) into the same columns),
+//   partial l, P codes -> st.shared into P buffer g%2 -> wait for PV_t(g-1)
+//   (barPV) -> rescale its 64 columns of O_t if a row maximum moved ->
+//   arrive barP.
+// The two halves of a row need no exchange per tile: the maximum is
+// computed redundantly, the partial sums l share every alpha and are added
+// once at the end of the item.
+// The MMA issuer of tile t, per KV tile g: S_t(g+1) once barSfree_t(g) (and
+// K(g+1)), then PV_t(g) once barP_t(g) (and V(g)).  A K stage is released
+// after both tiles' S MMAs of it, a V stage after both PVs; Q after both S
+// of an item's last tile (each barrier counts one commit per issuer).  None
+// of these events waits on an MMA issued after it, so the fixed order cannot
+// deadlock; every wait is bounded.
+#pragma once
+
+#include "attention.cuh"
+#include "device.cuh"
+
+namespace fqa {
+
+#ifndef FQA_PINGPONG
+#define FQA_PINGPONG 0
+#endif
+// 1: the two Q tiles' warpgroups take turns for their exponential loops.
+// Off by default: with four softmax warps per sub-partition the MUFU units
+// stay busier when all of them run freely (737 us against 830 us on the
+// 8704-token, 24-head workload).
+constexpr bool kPingPong = FQA_PINGPONG != 0;
+
+
+constexpr int kF8Threads = 640;
+// warp indices: Q/K producer, MMA issuer of tile 0 (and TMEM owner), V
+// producer, MMA issuer of tile 1
+constexpr int kF8Producer = 16, kF8Mma = 17, kF8ProducerV = 18, kF8Mma1 = 19;
+
+struct F8Traits {
+  static constexpr int kTileBytes = 128 * 128;                  // E4M3, 128 rows x 128 B
+  static constexpr int kStages = 3;
+  static constexpr uint32_t kIdescS = make_idesc(0, 0, 128, 128, 0);
+  static constexpr uint32_t kIdescPV = make_idesc(0, 0, 128, 128, 1);
+  static constexpr int kOffQ = 0;                                // Q0, Q1
+  static constexpr int kOffK = kOffQ + 2 * kTileBytes;
+  static constexpr int kOffV = kOffK + kStages * kTileBytes;
+  static constexpr int kOffP = kOffV + kStages * kTileBytes;     // [tile][buffer]
+  static constexpr int kOffL = kOffP + 4 * kTileBytes;          // [item parity][tile][half][row]
+  static constexpr int kOffBar = kOffL + 2 * 2 * 2 * 128 * 4;
+  // fullK, fullV, emptyK, emptyV [kStages]; barQ, barQfree; barS, barSfree,
+  // barP, barPV, barTurn, barDrain, barL [2 each]
+  static constexpr int kNumBars = 4 * kStages + 2 + 14;
+  static constexpr int kSmemBytes = kOffBar + 8 * kNumBars + 16 + 1024;
+};
+
+struct F8Item {
+  int b, h, qp;
+};
+
+__device__ __forceinline__ F8Item f8_item(int item, int H, int npairs) {
+  F8Item w;
+  w.qp = item % npairs;
+  const int bh = item / npairs;
+  w.h = bh % H;
+  w.b = bh / H;
+  return w;
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Maximum of 32 raw binary32 scores (two independent fmax3 chains).
+__device__ __forceinline__ float max32(const uint32_t (&u)[32]) {
+  float c0 = fmax3(__uint_as_float(u[0]), __uint_as_float(u[1]), __uint_as_float(u[2]));
+  float c1 = fmax3(__uint_as_float(u[16]), __uint_as_float(u[17]), __uint_as_float(u[18]));
+#pragma unroll
+  for (int e = 3; e < 15; e += 2) {
+    c0 = fmax3(c0, __uint_as_float(u[e]), __uint_as_float(u[e + 1]));
+    c1 = fmax3(c1, __uint_as_float(u[16 + e]), __uint_as_float(u[16 + e + 1]));
+  }
+  return fmax3(c0, __uint_as_float(u[15]), fmaxf(c1, __uint_as_float(u[31])));
+}
+
+__global__ void __launch_bounds__(kF8Threads, 1)
+    attn_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+  using T = F8Traits;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sQ = smem + T::kOffQ;
+  uint8_t* sK = smem + T::kOffK;
+  uint8_t* sV = smem + T::kOffV;
+  uint8_t* sP = smem + T::kOffP;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + T::kOffBar);
+  uint64_t* fullK = bars;
+  uint64_t* fullV = bars + T::kStages;
+  uint64_t* emptyK = bars + 2 * T::kStages;   // K(g) read by both S MMAs
+  uint64_t* emptyV = bars + 3 * T::kStages;   // V(g) read by both PV MMAs
+  uint64_t* barQ = bars + 4 * T::kStages;
+  uint64_t* barQfree = barQ + 1;
+  uint64_t* barS = barQ + 2;       // [2] S_t complete
+  uint64_t* barSfree = barQ + 4;   // [2] S_t read by its warpgroup
+  uint64_t* barP = barQ + 6;       // [2] P_t in shared memory, O_t rescaled
+  uint64_t* barPV = barQ + 8;      // [2] PV_t complete
+  uint64_t* barTurn = barQ + 10;   // [2] exponential-loop turns
+  uint64_t* barDrain = barQ + 12;  // [2] error path: an issuer's MMAs completed
+  uint64_t* barL = barQ + 14;      // [2] both halves' row sums written
+  float* sL = reinterpret_cast<float*>(smem + T::kOffL);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + T::kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int N = p.N, nkv = N / kBlockN, nblk = N / 64;
+  const int npairs = (N + 2 * kBlockM - 1) / (2 * kBlockM);
+  const int nitems = p.B * p.H * npairs;
+  // this CTA's items and KV tiles (tile g = local item * nkv + j)
+  const int my_items = nitems > (int)blockIdx.x ? (nitems - 1 - (int)blockIdx.x) / gridDim.x + 1 : 0;
+  const int ntiles = my_items * nkv;
+  const float c_log2e = p.softmax_scale * 1.4426950408889634f;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < T::kStages; ++s) {
+      mbar_init(&fullK[s], 1);
+      mbar_init(&fullV[s], 1);
+      mbar_init(&emptyK[s], 2);              // one commit per MMA issuer
+      mbar_init(&emptyV[s], 2);
+    }
+    mbar_init(barQ, 1);
+    mbar_init(barQfree, 2);
+    mbar_init(&barDrain[0], 1);
+    mbar_init(&barDrain[1], 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&barS[t], 1);
+      mbar_init(&barSfree[t], 2 * kBlockM);
+      mbar_init(&barP[t], 2 * kBlockM);
+      mbar_init(&barPV[t], 1);
+      mbar_init(&barTurn[t], 2 * kBlockM);
+      mbar_init(&barL[t], 2 * kBlockM);
+    }
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == kF8Mma) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == kF8Producer || warp == kF8ProducerV) {
+    // ------------------------------------------------ TMA producers: Q and
+    // K (warp kF8Producer), V (warp kF8ProducerV); each stage of K is
+    // refilled as soon as both S MMAs read it, each stage of V once both PVs
+    // did
+    if (lane == 0) {
+      const bool is_k = warp == kF8Producer;
+      const CUtensorMap* tm = is_k ? &tmK : &tmV;
+      uint64_t* full = is_k ? fullK : fullV;
+      uint64_t* empty = is_k ? emptyK : emptyV;
+      uint8_t* ring = is_k ? sK : sV;
+      if (is_k) tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(tm);
+      int g = 0, pending = 0;
+      bool ok = true;
+      for (int it = 0; ok && it < my_items; ++it) {
+        const F8Item w = f8_item((int)blockIdx.x + it * (int)gridDim.x, p.H, npairs);
+        const int head_row = (w.b * p.H + w.h) * N;
+        if (is_k) {
+          if (it > 0 && !(ok = mbar_wait(barQfree, (it - 1) & 1, abort_flag, p.status))) break;
+          mbar_arrive_expect_tx(barQ, 2 * T::kTileBytes);
+          tma_load_2d(sQ, &tmQ, barQ, 0, head_row + w.qp * 2 * kBlockM);
+          tma_load_2d(sQ + T::kTileBytes, &tmQ, barQ, 0, head_row + w.qp * 2 * kBlockM + kBlockM);
+        }
+        for (int j = 0; j < nkv; ++j, ++g) {
+          const int s = g % T::kStages, r = g / T::kStages;
+          if (!(ok = mbar_wait(&empty[s], (r & 1) ^ 1, abort_flag, p.status))) break;
+          mbar_arrive_expect_tx(&full[s], T::kTileBytes);
+          tma_load_2d(ring + s * T::kTileBytes, tm, &full[s], 0, head_row + j * kBlockN);
+          pending = g + 1;
+        }
+      }
+      if (*abort_flag) {
+        // let every copy this thread started land before the CTA exits
+        for (int q = (pending > T::kStages ? pending - T::kStages : 0); q < pending; ++q)
+          mbar_wait_drain(&full[q % T::kStages], (q / T::kStages) & 1);
+      }
+    }
+  } else if (warp == kF8Mma || warp == kF8Mma1) {
+    // ------------------------------------------------ MMA issuers, one per Q
+    // tile: an issuing thread is held for about as long as the tensor core
+    // takes for the MMA ahead of it, so each tile gets its own
+    if (lane == 0) {
+      // This thread shares its sub-partition with four softmax warps, so the
+      // issue path is kept short: descriptors are built once (a stage or a
+      // buffer only moves the start address, the low field, in 16-byte
+      // units) and the stage, phase and item counters advance without
+      // divisions.
+      const int t = warp == kF8Mma ? 0 : 1;
+      const uint64_t dQ = make_sdesc_sw128(smem_u32(sQ) + t * T::kTileBytes, 16, 1024);
+      const uint64_t dK0 = make_sdesc_sw128(smem_u32(sK), 16, 1024);
+      const uint64_t dV0 = make_sdesc_sw128(smem_u32(sV), 16384, 1024);
+      const uint64_t dP0 = make_sdesc_sw128(smem_u32(sP) + 2 * t * T::kTileBytes, 16, 1024);
+      constexpr uint64_t kTileStep = T::kTileBytes >> 4;
+      const uint32_t tS = tmem + 128u * t, tO = tmem + 256u + 128u * t;
+      bool ok = true;
+      // S_t(g) = Q_t K(g)^T for the tile at stage sk (phase bit kph, column
+      // block jk of item ik); commits barS_t, this issuer's share of the K
+      // stage release and, after an item's last KV tile, of barQfree
+      int sk = 0, jk = 0, ik = 0;
+      uint32_t kph = 0;
+      auto issue_s = [&]() -> bool {
+        if (jk == 0 && !mbar_wait(barQ, ik & 1, abort_flag, p.status)) return false;
+        if (!mbar_wait(&fullK[sk], kph, abort_flag, p.status)) return false;
+        tc_fence_after();
+        const uint64_t dK = dK0 + kTileStep * (uint64_t)sk;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)              // 32 keys' worth of K per step: +32 B
+          mma_f8_ss(tS, dQ + 2 * k, dK + 2 * k, T::kIdescS, k > 0);
+        tc_commit(&barS[t]);
+        tc_commit(&emptyK[sk]);
+        if (jk == nkv - 1) tc_commit(barQfree);
+        if (++sk == T::kStages) { sk = 0; kph ^= 1u; }
+        if (++jk == nkv) { jk = 0; ++ik; }
+        return true;
+      };
+      // O_t (+)= P_t(g) V(g) for the tile at stage sv (phase vph, column
+      // block jv), P buffer pb; commits barPV_t and this issuer's share of
+      // the V stage release
+      int sv = 0, jv = 0;
+      uint32_t vph = 0, pb = 0;
+      auto issue_pv = [&]() -> bool {
+        if (!mbar_wait(&fullV[sv], vph, abort_flag, p.status)) return false;
+        tc_fence_after();
+        const uint64_t dP = dP0 + kTileStep * (uint64_t)pb;
+        const uint64_t dV = dV0 + kTileStep * (uint64_t)sv;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)              // 32 keys per step: P +32 B, V +32 rows
+          mma_f8_ss(tO, dP + 2 * k, dV + 256 * k, T::kIdescPV, jv > 0 || k > 0);
+        tc_commit(&barPV[t]);
+        tc_commit(&emptyV[sv]);
+        if (++sv == T::kStages) { sv = 0; vph ^= 1u; }
+        if (++jv == nkv) jv = 0;
+        pb ^= 1u;
+        return true;
+      };
+      // per KV tile g: S_t(g+1) once the warpgroups of tile t have read
+      // S_t(g), then PV_t(g) once their P_t(g) landed
+      if (ntiles > 0) ok = issue_s();
+      for (int g = 0; ok && g < ntiles; ++g) {
+        if (g + 1 < ntiles) {
+          if (!(ok = mbar_wait(&barSfree[t], g & 1, abort_flag, p.status))) break;
+          if (!(ok = issue_s())) break;
+        }
+        if (!(ok = mbar_wait(&barP[t], g & 1, abort_flag, p.status))) break;
+        if (!(ok = issue_pv())) break;
+      }
+      if (!ok) {
+        // let the MMAs this thread issued finish before TMEM is released
+        tc_commit(&barDrain[t]);
+        mbar_wait_drain(&barDrain[t], 0);
+      }
+    }
+    __syncwarp();
+  } else if (warp < 16) {
+    // ------------------------------------------------ softmax warpgroups
+    const int t = warp >> 3;                     // Q tile of the pair
+    const int hf = (warp >> 2) & 1;              // half of the keys: [64hf, 64hf+64)
+    const int r = threadIdx.x & 127;             // row in tile == TMEM lane
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + 128u * t + lane_off, tO = tmem + 256u + 128u * t + lane_off;
+    // this thread's half row of the two P buffers; 16-byte chunk c of the
+    // row sits at c ^ (r % 8)
+    const uint32_t prow = smem_u32(sP) + (uint32_t)(2 * t) * T::kTileBytes + (uint32_t)r * 128u;
+    const uint32_t sw = (uint32_t)(r & 7);
+    int g = 0;                                   // KV tile counter (global over items)
+    bool ok = true;
+    for (int it = 0; ok && it < my_items; ++it) {
+      const F8Item w = f8_item((int)blockIdx.x + it * (int)gridDim.x, p.H, npairs);
+      const size_t head = (size_t)w.b * p.H + w.h;
+      const int qrow = w.qp * 2 * kBlockM + t * kBlockM + r;     // row within the head
+      const float* skp = p.sk + head * nblk;
+      const float* svp = p.sv + head * nblk;
+      const float svmax = p.sv_max[head];
+      const float a_row = p.sq[head * nblk + min(qrow, N - 1) / 64];
+      float sk0 = __ldg(skp), sk1 = __ldg(skp + 1), svh = __ldg(svp + hf);
+      float m = -INFINITY, l = 0.0f;
+      for (int j = 0; j < nkv; ++j, ++g) {
+        // block constants of this tile; the next tile's are loaded ahead
+        const float a0 = a_row * (sk0 * c_log2e), a1 = a_row * (sk1 * c_log2e);
+        const float ah = hf ? a1 : a0;
+        const float cpv = svmax > 0.0f ? 448.0f * (svh / svmax) : 0.0f;
+        if (j + 1 < nkv) {
+          sk0 = __ldg(skp + 2 * j + 2);
+          sk1 = __ldg(skp + 2 * j + 3);
+          svh = __ldg(svp + 2 * j + 2 + hf);
+        }
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(&barS[t], g & 1, abort_flag, p.status)))) break;
+        tc_fence_after();
+        // raw maxima of the other half (its scores are not kept) and of this
+        // half; the first 32 of this half's scores stay in registers, the
+        // other 32 are read again when the exponential loop gets to them.
+        // One 32-column load in flight besides sr keeps the registers low.
+        uint32_t sr[32];
+        float mo, mh;
+        {
+          const uint32_t oc = 64u * (uint32_t)(hf ^ 1), mc = 64u * (uint32_t)hf;
+          uint32_t v[32];
+          tmem_ld32(tS + oc, v);
+          tmem_ld32(tS + mc, sr);
+          tmem_wait_ld();
+          mo = max32(v);
+          tmem_ld32(tS + oc + 32u, v);
+          tmem_wait_ld();
+          mo = fmaxf(mo, max32(v));
+          tmem_ld32(tS + mc + 32u, v);
+          tmem_wait_ld();
+          mh = fmaxf(max32(sr), max32(v));
+        }
+        // raw maxima of keys [0,64) and [64,128); the scales are >= 0 and
+        // rounding is monotone, so the tile max of x = S * a (rounded toward
+        // zero) is the rounded product of the raw max
+        const float h0 = hf ? mo : mh, h1 = hf ? mh : mo;
+        const float m_new = fmaxf(m, fmaxf(__fmul_rz(h0, a0), __fmul_rz(h1, a1)));
+        const float alpha = ex2_approx(m - m_new);
+        const float2 nm2 = make_float2(-m_new, -m_new);
+        const float2 a2 = make_float2(ah, ah);
+        if (kPingPong && (t == 1 || g > 0)) {
+          // turn k of tile 1 follows turn k of tile 0
+          const uint32_t par = (t == 0) ? ((g - 1) & 1) : (g & 1);
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(&barTurn[t], par, abort_flag, p.status)))) break;
+        }
+        float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        const uint32_t pbuf = prow + (uint32_t)(g & 1) * T::kTileBytes;
+        const float2 c2 = make_float2(cpv, cpv);
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {               // 32 keys per chunk
+          if (ch == 1) {
+            tmem_ld32(tS + 64u * (uint32_t)hf + 32u, sr);
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(&barSfree[t]);           // S_t(g+1) may overwrite these columns
+          }
+          uint32_t pw[8];
+#pragma unroll
+          for (int w4 = 0; w4 < 8; ++w4) {
+            // x = S * a rounded once, toward zero: a rounding ptxas cannot
+            // fuse into the next step, fma(x, 1, -m), so the row maximum gets
+            // p = 1 exactly and x - m is exact near the maximum
+            const uint32_t* u = &sr[4 * w4];
+            const float2 x01 = f2_mul_rz(make_float2(__uint_as_float(u[0]), __uint_as_float(u[1])), a2);
+            const float2 x23 = f2_mul_rz(make_float2(__uint_as_float(u[2]), __uint_as_float(u[3])), a2);
+            const int e = 16 * ch + 2 * w4;
+            // pairs with (index % 8) < kPolyPer8 take the FMA-pipe exp2
+            const float2 p01 = (e % 8) < kPolyPer8 ? exp2_pair<true>(x01, nm2) : exp2_pair<false>(x01, nm2);
+            const float2 p23 = ((e + 1) % 8) < kPolyPer8 ? exp2_pair<true>(x23, nm2)
+                                                         : exp2_pair<false>(x23, nm2);
+            ls[0] = f2_add(ls[0], p01);
+            ls[1] = f2_add(ls[1], p23);
+            const float2 q01 = f2_mul(p01, c2), q23 = f2_mul(p23, c2);
+            pw[w4] = e4m3x4(q01.x, q01.y, q23.x, q23.y);
+          }
+          const uint32_t c0 = (uint32_t)(4 * hf + 2 * ch);
+          st_shared_v4(pbuf + ((c0 ^ sw) << 4), pw[0], pw[1], pw[2], pw[3]);
+          st_shared_v4(pbuf + (((c0 + 1) ^ sw) << 4), pw[4], pw[5], pw[6], pw[7]);
+        }
+        if (kPingPong) mbar_arrive(&barTurn[t ^ 1]);   // hand the turn to the other tile
+        const float2 l2 = f2_add(ls[0], ls[1]);
+        if (j > 0) {
+          // O_t holds PV_t(g-1) once it completed; rescale this half's
+          // columns if a row maximum moved
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(&barPV[t], (g - 1) & 1, abort_flag, p.status)))) break;
+          tc_fence_after();
+          if (__any_sync(0xffffffffu, m_new != m)) {
+            const float2 al2 = make_float2(alpha, alpha);
+#pragma unroll 1
+            for (int c = 0; c < 2; ++c) {
+              uint32_t o[32];
+              const uint32_t col = 64u * (uint32_t)hf + 32u * (uint32_t)c;
+              tmem_ld32(tO + col, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; e += 2) {
+                float2 v = f2_mul(make_float2(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), al2);
+                o[e] = __float_as_uint(v.x);
+                o[e + 1] = __float_as_uint(v.y);
+              }
+              tmem_st32(tO + col, o);
+            }
+            tmem_wait_st();
+          }
+        }
+        l = l * alpha + (l2.x + l2.y);
+        m = m_new;
+        fence_proxy_async_smem();                // P stores -> the MMA's operand reads
+        tc_fence_before();
+        mbar_arrive(&barP[t]);
+      }
+      if (!ok) break;
+      // ------------------------------------------------ epilogue: this half's columns
+      float* lx = sL + ((it & 1) * 2 + t) * 2 * 128;
+      lx[hf * 128 + r] = l;
+      mbar_arrive(&barL[t]);
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(&barL[t], it & 1, abort_flag, p.status)))) break;
+      const float l_row = lx[r] + lx[128 + r];
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(&barPV[t], (g - 1) & 1, abort_flag, p.status)))) break;
+      tc_fence_after();
+      const bool store = qrow < N;
+      const float fin = (svmax / 448.0f) / l_row;
+      const size_t orow = head * N + (size_t)qrow;
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        uint32_t o[32];
+        const int col = 64 * hf + 32 * c;
+        tmem_ld32(tO + (uint32_t)col, o);
+        tmem_wait_ld();
+        if (!store) continue;
+        if (p.out_f32) {
+          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow * 128 + col);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            dst[e] = make_float4(__uint_as_float(o[4 * e]) * fin, __uint_as_float(o[4 * e + 1]) * fin,
+                                 __uint_as_float(o[4 * e + 2]) * fin,
+                                 __uint_as_float(o[4 * e + 3]) * fin);
+        } else {
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + orow * 128 + col);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            uint32_t w4[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              __nv_bfloat162 pb = __floats2bfloat162_rn(__uint_as_float(o[8 * e + 2 * u]) * fin,
+                                                        __uint_as_float(o[8 * e + 2 * u + 1]) * fin);
+              w4[u] = *reinterpret_cast<uint32_t*>(&pb);
+            }
+            dst[e] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          }
+        }
+      }
+      // the next item's first PV overwrites O_t only after this warpgroup's
+      // next barP arrival, which comes after these loads
+      tc_fence_before();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kF8Mma) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace fqa

@@ -11,6 +11,7 @@
 
 #include "../../include/fqa.h"
 #include "attention.cuh"
+#include "attention_fp8.cuh"
 #include "attention_ws.cuh"
 #include "device.cuh"
 #include "quantize.cuh"
@@ -130,6 +131,26 @@ static fqa_status launch_attention_ws(const void* q, const void* k, const void* 
   return launch_status();
 }
 
+// FP8: persistent launch of the shared-memory-P kernel, one CTA per SM (or
+// per work item, if fewer).
+static fqa_status launch_attention_fp8(const void* q, const void* k, const void* v,
+                                       const AttnParams& prm, cudaStream_t stream) {
+  const uint64_t rows = (uint64_t)prm.B * prm.H * prm.N;
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap(&tq, q, true, rows) || !make_tmap(&tk, k, true, rows) ||
+      !make_tmap(&tv, v, true, rows))
+    return FQA_ERR_CUDA;
+  if (cudaFuncSetAttribute(attn_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           F8Traits::kSmemBytes) != cudaSuccess)
+    return FQA_ERR_CUDA;
+  const int items = prm.B * prm.H * ((prm.N + 2 * kBlockM - 1) / (2 * kBlockM));
+  const int sms = num_sms();
+  if (sms <= 0) return FQA_ERR_CUDA;
+  const int grid = items < sms ? items : sms;
+  attn_fp8_kernel<<<grid, kF8Threads, F8Traits::kSmemBytes, stream>>>(tq, tk, tv, prm);
+  return launch_status();
+}
+
 }  // namespace fqa
 
 using namespace fqa;
@@ -242,7 +263,7 @@ fqa_status fqa_attention_fp8(const void* q8, const void* k8, const void* v8, con
   uint32_t* status = status_ptr(&st);
   if (!status) return st;
   AttnParams prm{B, H, N, softmax_scale, sq, sk, sv, sv_max, out, out_dtype == FQA_OUT_F32, status};
-  return launch_attention_ws<true>(q8, k8, v8, prm, static_cast<cudaStream_t>(cuda_stream));
+  return launch_attention_fp8(q8, k8, v8, prm, static_cast<cudaStream_t>(cuda_stream));
 }
 
 fqa_status fqa_attention_bf16(const void* q, const void* k, const void* v, int B, int H, int N,
