@@ -36,7 +36,7 @@ NOMINAL_FP8_TFLOPS = 4500.0
 NOMINAL_BF16_TFLOPS = 2250.0
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = ["quantized_fp8_attention_b200/csrc/attention.cuh",
-                  "quantized_fp8_attention_b200/csrc/attention_ws.cuh",
+                  "quantized_fp8_attention_b200/csrc/attention_fp8.cuh",
                   "quantized_fp8_attention_b200/csrc/device.cuh"]
 
 
@@ -319,7 +319,7 @@ def run_fqa(args, rank: int, world: int):
                    "step": "fqa_quantize + fqa_attention_fp8",
                    "l2": "inputs larger than L2 (BF16 Q,K,V = %.0f MB per step)" % (3 * 2 * B * H * N * d / 1e6),
                    "parallelism": f"dp{world} (independent batches)"},
-        "roofline": {"bound": "tensor", "kernel": "attn_ws_kernel<true> (FP8)", "achieved": attn_tflops,
+        "roofline": {"bound": "tensor", "kernel": "attn_fp8_kernel", "achieved": attn_tflops,
                      "peak": fp8_peak, "unit": "TFLOP/s", "frac": attn_tflops / fp8_peak,
                      "peak_source": f"{pk_kind}: 2 x bf16_tflops (burst) of MEASURED_PEAKS.json",
                      "frac_of_nominal_4500": attn_tflops / NOMINAL_FP8_TFLOPS,
@@ -330,7 +330,7 @@ def run_fqa(args, rank: int, world: int):
                       "frac_of_nominal_2250": bf16_tflops / NOMINAL_BF16_TFLOPS},
         "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        # per step: quantize_fused_kernel + attn_ws_kernel<true> (plus one
+        # per step: quantize_fused_kernel + attn_fp8_kernel (plus one
         # 16-byte cudaMemsetAsync of the quantizer's counters)
         "gpu_launches": 2 * K,
         "clocks": clk.summary(),
@@ -342,8 +342,8 @@ def run_fqa(args, rank: int, world: int):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="fqa", choices=["fqa", "reference"])
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
