@@ -129,6 +129,24 @@ def host_inputs(w, rank: int):
     return synth.generate(wr), wr
 
 
+def max_over_ranks(x: float, device, world: int) -> float:
+    """The maximum of a per-rank float over all ranks (the job's time is its
+    slowest rank's); a plain value when world == 1."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(flops_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank processes flops_per_rank per step (weak
+    scaling), the step takes the slowest rank's time."""
+    return flops_per_rank * world / (ms_per_step * 1e-3) / 1e12
+
+
 # ------------------------------------------------------------ CPU baseline
 
 def oracle_sample(w, g, heads, rows):
@@ -250,11 +268,8 @@ def run_fqa(args, rank: int, world: int):
     if st != fqa.FQA_OK:
         raise RuntimeError(f"device status {flags:#x} after the timed steps")
 
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_per_step = float(t.item()) / K
-    value = flops * world / (ms_per_step * 1e-3) / 1e12
+    ms_per_step = max_over_ranks(total_ms, dev, world) / K
+    value = job_tflops(flops, world, ms_per_step)
 
     # BF16 comparison path (a9), same inputs
     for _ in range(3):
@@ -291,10 +306,7 @@ def run_fqa(args, rank: int, world: int):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    te = torch.tensor([e0.elapsed_time(e1) / Ke], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_ms = float(te.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / Ke, dev, world)
 
     if rank != 0:
         return
@@ -328,7 +340,7 @@ def run_fqa(args, rank: int, world: int):
                       "frac_of_hbm": quant_gbs / pk["hbm_gbs"], "hbm_peak_gbs": pk["hbm_gbs"]},
         "bf16_path": {"ms": bf16_ms, "tflops": bf16_tflops, "frac_of_bf16_peak": bf16_tflops / bf16_peak,
                       "frac_of_nominal_2250": bf16_tflops / NOMINAL_BF16_TFLOPS},
-        "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "e2e": {"value": job_tflops(flops, world, e2e_ms), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         # per step: quantize_fused_kernel + attn_fp8_kernel (plus one
         # 16-byte cudaMemsetAsync of the quantizer's counters)
