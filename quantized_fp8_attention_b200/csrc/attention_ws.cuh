@@ -1,10 +1,8 @@
-// attention_ws.cuh -- persistent, two-Q-tile attention forward on tcgen05.
-//
-// Same arithmetic as attention.cuh (the per-row rule is restated there): FP8
-// scaled dot-product attention with Q, K, V as E4M3 codes and per-64-token
-// block scales ("NVIDIA RTX AI optimiert FLUX.1 fuer Bilddaten mit niedriger
-// Genauigkeit", SDPA quantization paragraph), or the unquantized BF16 path
-// ("FLUX 3 Image Klein Base", section "왜 이런 차이가 나나").
+// attention_ws.cuh -- persistent, two-Q-tile BF16 attention forward on
+// tcgen05: the unquantized comparison path ("FLUX 3 Image Klein Base",
+// section "왜 이런 차이가 나나": VANILLA BF16 attention on B200), with the
+// per-row online softmax of attention.cuh minus the scales and the P
+// quantization (P in BF16, out = O / l).
 //
 // Organisation (one CTA per SM, persistent over work items):
 //   work item   = (b, h, pair of 128-row Q tiles); items taken round-robin
@@ -14,13 +12,16 @@
 //   warp 9      TMEM allocator and single-thread tcgen05.mma issuer
 //   warps 10-11 idle
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512);
-// P_t overwrites the top of S_t once softmax t holds S_t in registers.
+// P_t (BF16, 64 columns) overwrites the top of S_t once softmax t holds S_t
+// in registers.  A BF16 tile row is 256 B: every tile is two 64-column
+// halves of 128-byte-swizzled rows.
 // MMA issue order per KV tile j:  PV0(j), S0(j+1), PV1(j), S1(j+1)  -- the
 // tensor cores work on one tile while the other tile's softmax runs, and each
 // S_t(j+1) is issued after the PV_t(j) that reads P_t(j) from the same TMEM
 // columns (tcgen05.mma operations of one thread execute in issue order).  The
 // commit that signals S_t(j+1) also covers PV_t(j), so once softmax t sees
-// S_t(j+1) it may rescale O_t.
+// S_t(j+1) it may rescale O_t.  The two softmax warpgroups take turns for
+// their exponential loops.
 #pragma once
 
 #include "attention.cuh"
@@ -31,15 +32,13 @@ namespace fqa {
 constexpr int kWsThreads = 384;
 constexpr int kPairRows = 2 * kBlockM;
 
-template <bool kFP8>
-struct WsTraits {
-  static constexpr int kElt = kFP8 ? 1 : 2;
-  static constexpr int kTileBytes = kBlockM * kHeadDim * kElt;
-  static constexpr int kStages = kFP8 ? 3 : 2;
-  static constexpr int kKStep = kFP8 ? 32 : 16;
+struct BfTraits {
+  static constexpr int kTileBytes = kBlockM * kHeadDim * 2;       // BF16
+  static constexpr int kStages = 2;
+  static constexpr int kKStep = 16;                                // keys per MMA K step
   static constexpr int kSteps = 128 / kKStep;
-  static constexpr uint32_t kFmt = kFP8 ? 0u : 1u;
-  static constexpr uint32_t kPCol = kFP8 ? 96u : 64u;
+  static constexpr uint32_t kFmt = 1u;                             // BF16 operands
+  static constexpr uint32_t kPCol = 64u;                           // P_t in S_t columns [64,128)
   static constexpr uint32_t kIdescS = make_idesc(kFmt, kFmt, 128, 128, 0);
   static constexpr uint32_t kIdescPV = make_idesc(kFmt, kFmt, 128, 128, 1);
   static constexpr int kOffQ = 0;                                  // Q0, Q1
@@ -47,12 +46,9 @@ struct WsTraits {
   static constexpr int kOffV = kOffK + kStages * kTileBytes;
   static constexpr int kOffBar = kOffV + kStages * kTileBytes;
   // fullK, fullV, empty [kStages]; barQ, barQfree, barS[2], barP[2], barO[2],
-  // barSc[2], barTurn[2]
-  static constexpr int kNumBars = 3 * kStages + 12;
-  static constexpr int kOffScale = kOffBar + 8 * kNumBars + 16;
-  // per softmax warpgroup: two buffers (item parity) x {sk*c, 448*sv/svmax}
-  static constexpr int kScaleBytes = kFP8 ? 2 * 2 * 2 * kMaxScaleBlocks * 4 : 0;
-  static constexpr int kSmemBytes = kOffScale + kScaleBytes + 1024;
+  // barTurn[2]
+  static constexpr int kNumBars = 3 * kStages + 10;
+  static constexpr int kSmemBytes = kOffBar + 8 * kNumBars + 16 + 1024;
 };
 
 struct WsItem {
@@ -85,11 +81,10 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
       : "memory");
 }
 
-template <bool kFP8>
 __global__ void __launch_bounds__(kWsThreads, 1)
-    attn_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+    attn_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
-  using T = WsTraits<kFP8>;
+  using T = BfTraits;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -105,14 +100,12 @@ __global__ void __launch_bounds__(kWsThreads, 1)
   uint64_t* barS = barQ + 2;   // [2]
   uint64_t* barP = barQ + 4;   // [2]
   uint64_t* barO = barQ + 6;   // [2]
-  uint64_t* barSc = barQ + 8;  // [2] per-warpgroup scale tables written
-  uint64_t* barTurn = barQ + 10;  // [2] exponential-phase turns of the two softmax warpgroups
+  uint64_t* barTurn = barQ + 8;  // [2] exponential-phase turns of the two softmax warpgroups
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + T::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* scl = reinterpret_cast<float*>(smem + T::kOffScale);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int N = p.N, nkv = N / kBlockN, nblk = N / 64;
+  const int N = p.N, nkv = N / kBlockN;
   const int npairs = (N + kPairRows - 1) / kPairRows;
   const int nitems = p.B * p.H * npairs;
   const float c_log2e = p.softmax_scale * 1.4426950408889634f;
@@ -129,7 +122,6 @@ __global__ void __launch_bounds__(kWsThreads, 1)
       mbar_init(&barS[t], 1);
       mbar_init(&barP[t], kBlockM);
       mbar_init(&barO[t], 1);
-      mbar_init(&barSc[t], kBlockM);
       mbar_init(&barTurn[t], kBlockM);
     }
     *abort_flag = 0;
@@ -162,7 +154,7 @@ __global__ void __launch_bounds__(kWsThreads, 1)
           const int y = head_row + w.qp * kPairRows + t * kBlockM;
           uint8_t* dst = sQ + t * T::kTileBytes;
           tma_load_2d(dst, &tmQ, barQ, 0, y);
-          if constexpr (!kFP8) tma_load_2d(dst + 16384, &tmQ, barQ, 64, y);
+          tma_load_2d(dst + 16384, &tmQ, barQ, 64, y);
         }
         for (int j = 0; j < nkv; ++j, ++g) {
           const int s = g % T::kStages, r = g / T::kStages;
@@ -174,10 +166,8 @@ __global__ void __launch_bounds__(kWsThreads, 1)
           uint8_t* dv = sV + s * T::kTileBytes;
           tma_load_2d(dk, &tmK, &fullK[s], 0, y);
           tma_load_2d(dv, &tmV, &fullV[s], 0, y);
-          if constexpr (!kFP8) {
-            tma_load_2d(dk + 16384, &tmK, &fullK[s], 64, y);
-            tma_load_2d(dv + 16384, &tmV, &fullV[s], 64, y);
-          }
+          tma_load_2d(dk + 16384, &tmK, &fullK[s], 64, y);
+          tma_load_2d(dv + 16384, &tmV, &fullV[s], 64, y);
           pending = g + 1;
         }
       }
@@ -200,17 +190,14 @@ __global__ void __launch_bounds__(kWsThreads, 1)
       const uint32_t tO[2] = {tmem + 256, tmem + 384};
       int g = 0, it = 0, np[2] = {0, 0};
       bool ok = true;
-      auto kstep_kmajor = [](int k) -> uint64_t {     // K-major operand, bytes >> 4
-        return kFP8 ? (uint64_t)(2 * k) : (uint64_t)((k >> 2) * 1024 + (k & 3) * 2);
+      auto kstep_kmajor = [](int k) -> uint64_t {     // K-major operand, bytes >> 4:
+        return (uint64_t)((k >> 2) * 1024 + (k & 3) * 2);   // 32 B per step, 16 KB per half
       };
       auto issue_s = [&](int t, uint64_t dK) {
 #pragma unroll
         for (int k = 0; k < T::kSteps; ++k) {
           const uint64_t off = kstep_kmajor(k);
-          if constexpr (kFP8)
-            mma_f8_ss(tS[t], dQ[t] + off, dK + off, T::kIdescS, k > 0);
-          else
-            mma_bf16_ss(tS[t], dQ[t] + off, dK + off, T::kIdescS, k > 0);
+          mma_bf16_ss(tS[t], dQ[t] + off, dK + off, T::kIdescS, k > 0);
         }
         tc_commit(&barS[t]);
       };
@@ -219,10 +206,7 @@ __global__ void __launch_bounds__(kWsThreads, 1)
         for (int k = 0; k < T::kSteps; ++k) {
           const uint32_t aP = tS[t] + T::kPCol + 8u * (uint32_t)k;
           const uint64_t off = (uint64_t)(k * T::kKStep * 128 / 16);   // kKStep keys x 128 B
-          if constexpr (kFP8)
-            mma_f8_ts(tO[t], aP, dV + off, T::kIdescPV, (acc || k > 0));
-          else
-            mma_bf16_ts(tO[t], aP, dV + off, T::kIdescPV, (acc || k > 0));
+          mma_bf16_ts(tO[t], aP, dV + off, T::kIdescPV, (acc || k > 0));
         }
       };
       auto dK_of = [&](int s_) { return make_sdesc_sw128(smem_u32(sK + s_ * T::kTileBytes), 16, 1024); };
@@ -283,22 +267,6 @@ __global__ void __launch_bounds__(kWsThreads, 1)
       const WsItem w = ws_item(item, p.H, npairs);
       const size_t head = (size_t)w.b * p.H + w.h;
       const int qrow = w.qp * kPairRows + t * kBlockM + r;    // row within the head
-      // this warpgroup's own per-64-key-block constants for the item's head
-      // (double-buffered by item parity; published through an mbarrier so
-      // the wait stays bounded)
-      float* skc = scl + (2 * t + (it & 1)) * 2 * kMaxScaleBlocks;
-      float* pvc = skc + kMaxScaleBlocks;
-      float a_row = 0.0f, svmax = 0.0f;
-      if constexpr (kFP8) {
-        svmax = p.sv_max[head];
-        for (int jb = r; jb < nblk; jb += kBlockM) {
-          skc[jb] = p.sk[head * nblk + jb] * c_log2e;
-          pvc[jb] = svmax > 0.0f ? 448.0f * (p.sv[head * nblk + jb] / svmax) : 0.0f;
-        }
-        a_row = p.sq[head * nblk + min(qrow, N - 1) / 64];
-        mbar_arrive(&barSc[t]);
-        if (!(ok = __all_sync(0xffffffffu, mbar_wait(&barSc[t], it & 1, abort_flag, p.status)))) break;
-      }
       float m = -INFINITY, l = 0.0f;
       for (int j = 0; j < nkv; ++j, ++ns) {
         if (!(ok = __all_sync(0xffffffffu, mbar_wait(&barS[t], ns & 1, abort_flag, p.status)))) break;
@@ -307,13 +275,7 @@ __global__ void __launch_bounds__(kWsThreads, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld32(tS + lane_off + 32u * c, sr[c]);
         tmem_wait_ld();
-        float a0, a1;
-        if constexpr (kFP8) {
-          a0 = a_row * skc[2 * j];
-          a1 = a_row * skc[2 * j + 1];
-        } else {
-          a0 = a1 = c_log2e;
-        }
+        const float a0 = c_log2e, a1 = c_log2e;
         // maxima of the raw scores per 64-key half (8 independent chains);
         // the scales are >= 0 and rounding is monotone, so the tile max of
         // x = S * a (rounded toward zero) is the rounded product of the max
@@ -351,29 +313,7 @@ __global__ void __launch_bounds__(kWsThreads, 1)
           if (!(ok = __all_sync(0xffffffffu, mbar_wait(&barTurn[t], par, abort_flag, p.status)))) break;
         }
         float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-        if constexpr (kFP8) {
-          const float cpv0 = pvc[2 * j], cpv1 = pvc[2 * j + 1];
-#pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {             // 32 keys per chunk
-            const float cc = (ch < 2) ? cpv0 : cpv1;
-            const float2 c2 = make_float2(cc, cc);
-            uint32_t pw[8];
-#pragma unroll
-            for (int w4 = 0; w4 < 8; ++w4) {
-              const int e = 16 * ch + 2 * w4;
-              // pairs with (index % 8) < kPolyPer8 take the FMA-pipe exp2
-              const float2 p01 = (e % 8) < kPolyPer8 ? exp2_pair<true>(X[e], nm2)
-                                                     : exp2_pair<false>(X[e], nm2);
-              const float2 p23 = ((e + 1) % 8) < kPolyPer8 ? exp2_pair<true>(X[e + 1], nm2)
-                                                           : exp2_pair<false>(X[e + 1], nm2);
-              ls[0] = f2_add(ls[0], p01);
-              ls[1] = f2_add(ls[1], p23);
-              const float2 q01 = f2_mul(p01, c2), q23 = f2_mul(p23, c2);
-              pw[w4] = e4m3x4(q01.x, q01.y, q23.x, q23.y);
-            }
-            tmem_st8(tS + lane_off + T::kPCol + 8u * ch, pw);
-          }
-        } else {
+        {
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch) {
             uint32_t pw[16];
@@ -419,7 +359,7 @@ __global__ void __launch_bounds__(kWsThreads, 1)
       if (!(ok = __all_sync(0xffffffffu, mbar_wait(&barO[t], it & 1, abort_flag, p.status)))) break;
       tc_fence_after();
       const bool store = qrow < N;
-      const float fin = kFP8 ? (svmax / 448.0f) / l : 1.0f / l;
+      const float fin = 1.0f / l;
       const size_t orow = head * N + (size_t)qrow;
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {

@@ -109,25 +109,22 @@ static int num_sms() {
   return g_dev[dev].num_sms;
 }
 
-// Persistent launch: one CTA per SM (or per work item, if fewer).
-template <bool kFP8>
-static fqa_status launch_attention_ws(const void* q, const void* k, const void* v,
-                                      const AttnParams& prm, cudaStream_t stream) {
-  using T = WsTraits<kFP8>;
+// BF16: persistent launch, one CTA per SM (or per work item, if fewer).
+static fqa_status launch_attention_bf16(const void* q, const void* k, const void* v,
+                                        const AttnParams& prm, cudaStream_t stream) {
   const uint64_t rows = (uint64_t)prm.B * prm.H * prm.N;
   CUtensorMap tq, tk, tv;
-  if (!make_tmap(&tq, q, kFP8, rows) || !make_tmap(&tk, k, kFP8, rows) ||
-      !make_tmap(&tv, v, kFP8, rows))
+  if (!make_tmap(&tq, q, false, rows) || !make_tmap(&tk, k, false, rows) ||
+      !make_tmap(&tv, v, false, rows))
     return FQA_ERR_CUDA;
-  auto kern = attn_ws_kernel<kFP8>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, T::kSmemBytes) !=
-      cudaSuccess)
+  if (cudaFuncSetAttribute(attn_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           BfTraits::kSmemBytes) != cudaSuccess)
     return FQA_ERR_CUDA;
   const int items = prm.B * prm.H * ((prm.N + kPairRows - 1) / kPairRows);
   const int sms = num_sms();
   if (sms <= 0) return FQA_ERR_CUDA;
   const int grid = items < sms ? items : sms;
-  kern<<<grid, kWsThreads, T::kSmemBytes, stream>>>(tq, tk, tv, prm);
+  attn_bf16_kernel<<<grid, kWsThreads, BfTraits::kSmemBytes, stream>>>(tq, tk, tv, prm);
   return launch_status();
 }
 
@@ -280,7 +277,7 @@ fqa_status fqa_attention_bf16(const void* q, const void* k, const void* v, int B
   if (!status) return st;
   AttnParams prm{B, H, N, softmax_scale, nullptr, nullptr, nullptr, nullptr, out,
                  out_dtype == FQA_OUT_F32, status};
-  return launch_attention_ws<false>(q, k, v, prm, static_cast<cudaStream_t>(cuda_stream));
+  return launch_attention_bf16(q, k, v, prm, static_cast<cudaStream_t>(cuda_stream));
 }
 
 fqa_status fqa_e4m3_encode(const float* x, uint8_t* out, size_t n, void* cuda_stream) {

@@ -194,3 +194,37 @@ def test_attention_rejects_bad_arguments():
     assert fqa.fqa_attention_fp8(t, t, t, s, s, s, sm, U.SCALE, out, 7) == fqa.FQA_ERR_INVALID_ARG
     tb = torch.zeros(1, 1, 128, 128, dtype=torch.bfloat16, device="cuda")
     assert fqa.fqa_attention_bf16(tb, tb, tb, -1.0, out, 0) == fqa.FQA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("B,H,N", [(2, 96, 128), (1, 200, 384)])
+def test_fp8_many_items_per_cta(B, H, N):
+    """More work items than SMs: with N = 128 every item has one KV tile, so
+    the per-item barriers (Q reload, PV completion, the halves' row sums)
+    turn over on every tile; with N = 384 the second Q tile of each item's
+    last pair lies beyond N.  Every row against the oracle."""
+    fqa = _fqa()
+    shape = (B, H, N, 128)
+    bits = {t: _gen(shape, 60 + i, 2.0) for i, t in enumerate("qkv")}
+    q, k, v = (U.to_device(bits[t]) for t in "qkv")
+    out = fqa.attention_fp8(fqa.quantize(q, k, v), U.SCALE, fqa.FQA_OUT_F32).cpu().numpy()
+    ref, amb, _ = oracle.attention_fp8(oracle.quantize(bits["q"], bits["k"], bits["v"]), U.SCALE,
+                                       with_ambiguity=True)
+    got = out.reshape(ref.shape)
+    m = U.metrics(got, ref)
+    assert m["mean_rel"] <= 2e-3, m
+    assert np.all(np.abs(got - ref) <= 1e-2 + amb)
+    assert fqa.fqa_debug_status()[0] == fqa.FQA_OK
+
+
+def test_bf16_many_items_per_cta():
+    """The BF16 path with more work items than SMs and one KV tile per item."""
+    fqa = _fqa()
+    shape = (2, 96, 128, 128)
+    bits = {t: _gen(shape, 70 + i) for i, t in enumerate("qkv")}
+    q, k, v = (U.to_device(bits[t]) for t in "qkv")
+    out = fqa.attention_bf16(q, k, v, U.SCALE, fqa.FQA_OUT_F32).cpu().numpy().astype(np.float64)
+    ex = oracle.attention_exact(bits["q"], bits["k"], bits["v"], U.SCALE)
+    got = out.reshape(ex.shape)
+    m = U.metrics(got, ex)
+    assert m["cos"] >= 0.9999 and m["mean_rel"] <= 1e-2, m
+    assert np.all(np.abs(got - ex) <= 2e-2 + 2.0 ** -8 * np.abs(ex))
