@@ -9,6 +9,8 @@ independently seeded batch; no data-path collective: weak scaling).
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fqa|reference]
 For N > 1 launch with torch.distributed.run (one rank per GPU).
+python bench.py --sweep prints one line per workload (quantizer, FP8 and BF16
+attention timed separately, at most 200 launches each) instead.
 """
 
 from __future__ import annotations
@@ -145,6 +147,91 @@ def job_tflops(flops_per_rank: int, world: int, ms_per_step: float) -> float:
     """Whole-job throughput: every rank processes flops_per_rank per step (weak
     scaling), the step takes the slowest rank's time."""
     return flops_per_rank * world / (ms_per_step * 1e-3) / 1e12
+
+
+def fp8_gemm_probe(dev):
+    """A library FP8 GEMM for context (cuBLASLt through torch._scaled_mm,
+    8192^3 E4M3 x E4M3 -> BF16, best of 10 after warm-up).  Not the roofline
+    denominator: that is the measured BF16 peak x the nominal FP8:BF16 ratio."""
+    import torch
+    n = 8192
+    try:
+        a = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn)
+        b = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn).t()
+        one = torch.ones((), device=dev)
+        for _ in range(3):
+            torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        best = float("inf")
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for _ in range(10):
+            e0.record()
+            torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+            e1.record()
+            torch.cuda.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        return {"tflops": 2 * n ** 3 / (best * 1e-3) / 1e12,
+                "how": "torch._scaled_mm 8192^3 e4m3 x e4m3 -> bf16, best of 10 (context only)"}
+    except Exception as exc:  # an FP8 GEMM the local torch build does not offer
+        return {"tflops": None, "how": f"unavailable: {type(exc).__name__}"}
+
+
+def run_sweep(args):
+    """One JSON line per workload: quantizer, FP8 attention and BF16 attention
+    each timed alone with CUDA events (the quantizer with an L2 flush before
+    every launch), at most 200 launches (about half a second) per kernel."""
+    import torch
+
+    import quantized_fp8_attention_b200 as fqa
+    from quantized_fp8_attention_b200 import build as fqa_build
+
+    fqa_build.build()
+    dev = torch.device("cuda", 0)
+    pk, pk_kind = peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for w in synth.WORKLOADS:
+        g = synth.generate(w)
+        q, k, v = (torch.from_numpy(g[t].view(np.int16)).view(torch.bfloat16).to(dev) for t in "qkv")
+        qz = fqa.alloc_quantized(w.B, w.H, w.N, dev)
+        ws = fqa.alloc_workspace(w.B, w.H, w.N, dev)
+        out = torch.empty(w.B, w.H, w.N, w.d, dtype=torch.bfloat16, device=dev)
+        scale = fqa.softmax_scale(w.d)
+
+        def timed(fn, reps, pre=None):
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize()
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(2 * reps)]
+            for i in range(reps):
+                if pre:
+                    pre()
+                e[2 * i].record()
+                fn()
+                e[2 * i + 1].record()
+            torch.cuda.synchronize()
+            return sum(e[2 * i].elapsed_time(e[2 * i + 1]) for i in range(reps)) / reps
+
+        fqa.quantize(q, k, v, out=qz, workspace=ws)
+        # about 0.5 s of each kernel, between 5 and 200 launches
+        reps = lambda tflops: min(200, max(5, int(0.5 / (w.flops / (tflops * 1e12)))))
+        ms_a = timed(lambda: fqa.attention_fp8(qz, scale, fqa.FQA_OUT_BF16, out=out), reps(1200))
+        ms_b = timed(lambda: fqa.attention_bf16(q, k, v, scale, fqa.FQA_OUT_BF16, out=out), reps(850))
+        ms_q = timed(lambda: fqa.quantize(q, k, v, out=qz, workspace=ws), 200, pre=lambda: flush.fill_(1))
+        st, flags = fqa.fqa_debug_status()
+        if st != fqa.FQA_OK:
+            raise RuntimeError(f"device status {flags:#x} on {w.name}")
+        fp8_peak = 2 * pk["bf16_tflops"]
+        qbytes = 9 * w.B * w.H * w.N * w.d
+        print(json.dumps({
+            "sweep": True, "workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+            "attention_fp8": {"ms": ms_a, "tflops": w.flops / ms_a / 1e9,
+                              "frac_of_fp8_peak": w.flops / ms_a / 1e9 / fp8_peak},
+            "attention_bf16": {"ms": ms_b, "tflops": w.flops / ms_b / 1e9,
+                               "frac_of_bf16_peak": w.flops / ms_b / 1e9 / pk["bf16_tflops"]},
+            "quantizer": {"ms": ms_q, "gbs": qbytes / ms_q / 1e6, "frac_of_hbm": qbytes / ms_q / 1e6 / pk["hbm_gbs"],
+                          "l2": "flushed before every launch"},
+            "peaks": pk_kind}), flush=True)
+        del q, k, v, qz, ws, out
+        torch.cuda.empty_cache()
 
 
 # ------------------------------------------------------------ CPU baseline
@@ -318,6 +405,7 @@ def run_fqa(args, rank: int, world: int):
     quant_gbs = quant_bytes / (quant_ms * 1e-3) / 1e9
     bf16_tflops = flops / (bf16_ms * 1e-3) / 1e12
     tr = traffic_per_launch()
+    probe = fp8_gemm_probe(dev)
     cpu = None
     if not args.no_cpu_baseline:
         cpu = cpu_baseline(w, g)
@@ -346,6 +434,7 @@ def run_fqa(args, rank: int, world: int):
         # 16-byte cudaMemsetAsync of the quantizer's counters)
         "gpu_launches": 2 * K,
         "clocks": clk.summary(),
+        "fp8_gemm_probe": probe,
         "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)
@@ -354,12 +443,16 @@ def run_fqa(args, rank: int, world: int):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--steps", type=int, default=1200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="fqa", choices=["fqa", "reference"])
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true", help="one line per workload instead of the step")
     args = ap.parse_args()
+    if args.sweep:
+        run_sweep(args)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if args.impl == "reference":
