@@ -38,8 +38,9 @@
  *  - Layouts are row-major and contiguous: [B, H, N, d] with d innermost.
  *  - v1 limits: d == 128; N a multiple of 128 (quantizer: of 64);
  *    1 <= N <= 65536; B, H >= 1, B*H <= 65535, B*H*N < 2^31; device pointers
- *    16-byte aligned (scale arrays 4-byte aligned); a finite softmax_scale > 0;
- *    outputs must not overlap inputs.
+ *    16-byte aligned (the block-scale arrays and sv_max 4-byte aligned; k_mean
+ *    16-byte aligned); a finite softmax_scale > 0; outputs must not overlap
+ *    inputs.
  *  - Errors: arguments are checked on the host before anything is launched;
  *    an argument error returns a status and launches nothing.  A launch
  *    failure returns FQA_ERR_CUDA.  Non-finite input values are outside the
@@ -171,6 +172,10 @@ FQA_API size_t fqa_quantize_noalloc_max_workspace_bytes(void);
  *   out_i = O * (sv_max / 448) / l
  * Scores use the smoothed K codes; smoothing leaves softmax unchanged because
  * q . k_mean is constant along a row.  sv_max == 0 gives out = 0.
+ * Evaluated in binary32: x = fl(S * a) rounded toward zero, then x - m, so
+ * the row maximum gets p = 1 exactly; a P code whose binary32 value lies
+ * within evaluation error of an E4M3 rounding midpoint may round either way.
+ * Enqueues one persistent kernel launch (one CTA per SM).
  *
  * out: [B,H,N,d] BF16 (FQA_OUT_BF16) or FP32 (FQA_OUT_F32).
  * softmax_scale: typically fl32(1/sqrt(d)).

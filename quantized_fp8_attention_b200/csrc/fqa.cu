@@ -189,10 +189,10 @@ fqa_status fqa_quantize(const void* q, const void* k, const void* v, int B, int 
   for (const void* p : ptrs)
     if (p == nullptr) return FQA_ERR_INVALID_ARG;
   if (workspace_bytes < fqa_quantize_workspace_bytes(B, H, N, d)) return FQA_ERR_INVALID_ARG;
-  const void* a16[] = {q, k, v, q8, k8, v8, workspace};
+  const void* a16[] = {q, k, v, q8, k8, v8, k_mean, workspace};   // k_mean: read by bulk copies
   for (const void* p : a16)
     if (!aligned(p, 16)) return FQA_ERR_MISALIGNED;
-  const void* a4[] = {sq, sk, sv, sv_max, k_mean};
+  const void* a4[] = {sq, sk, sv, sv_max};
   for (const void* p : a4)
     if (!aligned(p, 4)) return FQA_ERR_MISALIGNED;
   uint32_t* status = status_ptr(&st);

@@ -29,7 +29,8 @@ namespace fqa {
 //       K read last and marked evict-last in L2 for phase 3
 //   2   per (b, h): k_mean from the partials in block order; sv_max = max of
 //       the V unit scales (no atomics)
-//   3   K units -> smoothed codes and scales, newest units of 1b first
+//   3   K units -> smoothed codes and scales, newest units of 1b first (each
+//       unit's head mean row arrives with the unit)
 // Unit u = (b*H + h)*(N/64) + j is one 64-token block of one head: 16 KB of
 // contiguous BF16 per tensor.  Units are handed out through work queues
 // (counters the launch zeroes), so the SMs that stream faster take more.
@@ -149,7 +150,6 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantMinCtas) quantize_fused_k
   __shared__ uint64_t full[kMaxSlots];
   __shared__ int slot_unit[kMaxSlots];
   __shared__ float red[2 * kQuantWarps];
-  __shared__ float mu[kHeadDim];
   __shared__ int failed, abort_flag;
   const int t = threadIdx.x;
   const int nblk = N / kQBlock;
@@ -301,24 +301,21 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantMinCtas) quantize_fused_k
   }
   if (!grid_barrier(&ctr[kCtrBarrier], 2, status, &failed)) return;
 
-  // ---- phase 3: K codes, newest units of phase 1b first
-  int last_head = -1;
-  float mr[8];                                     // k_mean of this thread's 8 channels
-  run(kBlockBytes, queue(kCtrK3, true),
+  // ---- phase 3: K codes, newest units of phase 1b first.  Each slot holds
+  // the unit's K block and its head's k_mean row (512 B), loaded together.
+  constexpr int kSlot3 = kBlockBytes + kHeadDim * 4;
+  run(kSlot3, queue(kCtrK3, true),
       [&](int u, uint8_t* dst, uint64_t* bar) {
-        mbar_arrive_expect_tx(bar, kBlockBytes);
+        mbar_arrive_expect_tx(bar, kSlot3);
         bulk_load(dst, blk_ptr(k, u), kBlockBytes, bar, pol_first);
+        bulk_load(dst + kBlockBytes, k_mean + (size_t)(u / nblk) * kHeadDim, kHeadDim * 4, bar, pol_first);
       },
       [&](int u, const uint8_t* blk) {
-        const int head = u / nblk;
-        if (head != last_head) {                   // CTA-uniform
-          if (t < kHeadDim) mu[t] = __ldcg(k_mean + (size_t)head * kHeadDim + t);
-          __syncthreads();
-          // every chunk of this thread starts at channel 8t mod 128
+        // every chunk of this thread starts at channel 8t mod 128
+        const float* mu = reinterpret_cast<const float*>(blk + kBlockBytes) + ((8 * t) & (kHeadDim - 1));
+        float mr[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) mr[e] = mu[((8 * t) & (kHeadDim - 1)) + e];
-          last_head = head;
-        }
+        for (int e = 0; e < 8; ++e) mr[e] = mu[e];
         float x[kVals];
         chunks_to_f32(blk, x);
 #pragma unroll

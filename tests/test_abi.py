@@ -78,6 +78,7 @@ def test_quantize_validation(L):
     assert L.fqa_quantize(*args(wsb=16)) == 1
     assert L.fqa_quantize(*args(k=_p(0x10008))) == 3
     assert L.fqa_quantize(*args(sq=_p(0x10002))) == 3
+    assert L.fqa_quantize(*args(km=_p(0x10004))) == 3      # k_mean: 16-byte aligned
 
 
 def test_attention_validation(L):
