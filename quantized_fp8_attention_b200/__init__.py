@@ -156,6 +156,37 @@ def fqa_debug_status(stream=None):
 
 # ----------------------------------------------------- tensor-level API
 
+def _require(t, dtype: torch.dtype, name: str, shape=None) -> None:
+    """The C ABI takes contiguous device buffers of a fixed element type and
+    shape; anything else is refused here, before a pointer is passed on."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name}: expected a CUDA tensor, got one on {t.device}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: expected {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: expected a contiguous tensor")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _require_qkv(q, k, v, dtype: torch.dtype):
+    if not isinstance(q, torch.Tensor) or q.dim() != 4:
+        raise ValueError("q: expected a [B, H, N, 128] tensor")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _require(t, dtype, name, q.shape)
+    if q.device != k.device or q.device != v.device:
+        raise ValueError("q, k and v must be on the same device")
+    return tuple(q.shape)
+
+
+def _require_quantized(qz: "Quantized", B: int, H: int, N: int) -> None:
+    shapes = ((B, H, N, HEAD_DIM),) * 3 + ((B, H, N // 64),) * 3 + ((B, H), (B, H, HEAD_DIM))
+    for name, t, shape in zip(Quantized._fields, qz, shapes):
+        _require(t, torch.uint8 if name.endswith("8") else torch.float32, name, shape)
+
+
 class Quantized(NamedTuple):
     q8: torch.Tensor       # uint8 E4M3 codes [B,H,N,128]
     k8: torch.Tensor
@@ -184,21 +215,27 @@ def alloc_workspace(B: int, H: int, N: int, device) -> torch.Tensor:
 def quantize(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: Optional[Quantized] = None,
              workspace: Optional[torch.Tensor] = None, stream=None) -> Quantized:
     """BF16 [B,H,N,128] Q, K, V (CUDA, contiguous) -> Quantized."""
-    B, H, N, _ = q.shape
+    B, H, N, _ = _require_qkv(q, k, v, torch.bfloat16)
     if out is None:
         out = alloc_quantized(B, H, N, q.device)
+    _require_quantized(out, B, H, N)
     if workspace is None:
         workspace = alloc_workspace(B, H, N, q.device)
+    _require(workspace, workspace.dtype, "workspace")
     _check(fqa_quantize(q, k, v, *out, workspace, stream=stream), "fqa_quantize")
     return out
 
 
 def attention_fp8(qz: Quantized, softmax_scale: float, out_dtype: int = FQA_OUT_BF16,
                   out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    if not isinstance(qz.q8, torch.Tensor) or qz.q8.dim() != 4:
+        raise ValueError("qz.q8: expected a [B, H, N, 128] tensor")
     B, H, N, d = qz.q8.shape
+    _require_quantized(qz, B, H, N)
+    dt = torch.float32 if out_dtype == FQA_OUT_F32 else torch.bfloat16
     if out is None:
-        dt = torch.float32 if out_dtype == FQA_OUT_F32 else torch.bfloat16
         out = torch.empty(B, H, N, d, dtype=dt, device=qz.q8.device)
+    _require(out, dt, "out", (B, H, N, d))
     _check(fqa_attention_fp8(qz.q8, qz.k8, qz.v8, qz.sq, qz.sk, qz.sv, qz.sv_max, softmax_scale,
                              out, out_dtype, stream=stream), "fqa_attention_fp8")
     return out
@@ -207,10 +244,11 @@ def attention_fp8(qz: Quantized, softmax_scale: float, out_dtype: int = FQA_OUT_
 def attention_bf16(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, softmax_scale: float,
                    out_dtype: int = FQA_OUT_BF16, out: Optional[torch.Tensor] = None,
                    stream=None) -> torch.Tensor:
-    B, H, N, d = q.shape
+    B, H, N, d = _require_qkv(q, k, v, torch.bfloat16)
+    dt = torch.float32 if out_dtype == FQA_OUT_F32 else torch.bfloat16
     if out is None:
-        dt = torch.float32 if out_dtype == FQA_OUT_F32 else torch.bfloat16
         out = torch.empty(B, H, N, d, dtype=dt, device=q.device)
+    _require(out, dt, "out", (B, H, N, d))
     _check(fqa_attention_bf16(q, k, v, softmax_scale, out, out_dtype, stream=stream),
            "fqa_attention_bf16")
     return out
@@ -223,6 +261,7 @@ def fp8_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, softmax_sca
 
 
 def e4m3_encode(x: torch.Tensor, stream=None) -> torch.Tensor:
+    _require(x, torch.float32, "x")
     out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
     _check(fqa_e4m3_encode(x, out, stream=stream), "fqa_e4m3_encode")
     return out
