@@ -269,7 +269,10 @@ def run_reference(args, rank: int, world: int):
         return
     w = synth.workload(args.workload)
     g = synth.generate(w, heads=[(0, h) for h in range(2)])
-    rows = list(range(0, w.N, max(1, w.N // 256)))[:256]
+    # per-step sample sized so that the whole run stays within a few minutes:
+    # 256 strided query rows up to 50 steps, fewer beyond (at least 64)
+    n_rows = max(64, min(256, (256 * 50) // max(1, args.steps + args.warmup)))
+    rows = list(range(0, w.N, max(1, w.N // n_rows)))[:n_rows]
     heads = [(0, 0), (0, 1)]
     for _ in range(args.warmup):
         oracle_sample(w, g, heads, rows[:16])
