@@ -17,8 +17,10 @@ Parity status (see the tests under tests/test_oracle_*.py for the pins):
     bounds, hand-worked blocks).
   * Tiled attention skeleton: pinned (identity codec == exact softmax
     attention; FP64 brute force; invariants).
-  * P rounding rule E4M3(p * 448 * sv_J / sv_max): pinned only by hand-worked
-    cases of its own reading; the pages print no worked example.
+  * P rounding rule E4M3(p * 448 * sv_J / sv_max): pinned by hand-worked
+    cases and by an independent 40-digit re-evaluation of the whole rule
+    (tests/test_oracle_highprec.py); the rule itself is a reading, since the
+    pages print no worked example.
 """
 
 from __future__ import annotations
