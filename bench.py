@@ -234,6 +234,52 @@ def run_sweep(args):
         torch.cuda.empty_cache()
 
 
+def step_line(w, world: int, K: int, warmup: int, ms_per_step: float, attn_ms: float, quant_ms: float,
+              bf16_ms: float, e2e_ms: float, h2d: int, d2h: int, clocks: dict, probe, cpu, traffic,
+              pk: dict, pk_kind: str) -> dict:
+    """The benchmark's JSON line for workload w from the measured times (ms).
+    value and e2e are whole-job throughput (every rank runs its own batch);
+    roofline is for the FP8 attention kernel against 2 x the measured BF16
+    peak (the nominal FP8:BF16 ratio)."""
+    B, H, N, d = w.B, w.H, w.N, w.d
+    flops = w.flops
+    fp8_peak = 2.0 * pk["bf16_tflops"]            # FP8 dense = 2 x BF16 dense (nominal ratio)
+    bf16_peak = pk["bf16_tflops"]
+    attn_tflops = flops / (attn_ms * 1e-3) / 1e12
+    quant_bytes = 9 * B * H * N * d
+    quant_gbs = quant_bytes / (quant_ms * 1e-3) / 1e9
+    bf16_tflops = flops / (bf16_ms * 1e-3) / 1e12
+    return {
+        "metric": METRIC, "value": job_tflops(flops, world, ms_per_step), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": K, "warmup": warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 (fp32 accumulate)",
+        "data": "synthetic (seeded, FLUX-style token mix; see fqa_synth)",
+        "config": {"workload": w.name, "B": B, "H": H, "N": N, "d": d,
+                   "n_text": w.n_text, "n_ctx": w.n_ctx, "n_img": w.n_img,
+                   "step": "fqa_quantize + fqa_attention_fp8",
+                   "l2": "inputs larger than L2 (BF16 Q,K,V = %.0f MB per step)" % (3 * 2 * B * H * N * d / 1e6),
+                   "parallelism": f"dp{world} (independent batches)"},
+        "roofline": {"bound": "tensor", "kernel": "attn_fp8_kernel", "achieved": attn_tflops,
+                     "peak": fp8_peak, "unit": "TFLOP/s", "frac": attn_tflops / fp8_peak,
+                     "peak_source": f"{pk_kind}: 2 x bf16_tflops (burst) of MEASURED_PEAKS.json",
+                     "frac_of_nominal_4500": attn_tflops / NOMINAL_FP8_TFLOPS,
+                     "ms_per_launch": attn_ms, "traffic": traffic},
+        "quantizer": {"ms": quant_ms, "gbs": quant_gbs, "algorithmic_bytes": quant_bytes,
+                      "frac_of_hbm": quant_gbs / pk["hbm_gbs"], "hbm_peak_gbs": pk["hbm_gbs"]},
+        "bf16_path": {"ms": bf16_ms, "tflops": bf16_tflops, "frac_of_bf16_peak": bf16_tflops / bf16_peak,
+                      "frac_of_nominal_2250": bf16_tflops / NOMINAL_BF16_TFLOPS},
+        "e2e": {"value": job_tflops(flops, world, e2e_ms), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                "pipeline": "two device buffer sets; uploads, kernels and downloads on three streams"},
+        # per step: quantize_fused_kernel + attn_fp8_kernel (plus one
+        # 16-byte cudaMemsetAsync of the quantizer's counters)
+        "gpu_launches": 2 * K,
+        "clocks": clocks,
+        "fp8_gemm_probe": probe,
+        "cpu_baseline": cpu,
+    }
+
+
 # ------------------------------------------------------------ CPU baseline
 
 def oracle_sample(w, g, heads, rows):
@@ -359,7 +405,6 @@ def run_fqa(args, rank: int, world: int):
         raise RuntimeError(f"device status {flags:#x} after the timed steps")
 
     ms_per_step = max_over_ranks(total_ms, dev, world) / K
-    value = job_tflops(flops, world, ms_per_step)
 
     # BF16 comparison path (a9), same inputs
     for _ in range(3):
@@ -427,46 +472,10 @@ def run_fqa(args, rank: int, world: int):
     if rank != 0:
         return
     pk, pk_kind = peaks()
-    fp8_peak = 2.0 * pk["bf16_tflops"]            # FP8 dense = 2 x BF16 dense (nominal ratio)
-    bf16_peak = pk["bf16_tflops"]
-    attn_tflops = flops / (attn_ms * 1e-3) / 1e12
-    quant_bytes = 9 * B * H * N * d
-    quant_gbs = quant_bytes / (quant_ms * 1e-3) / 1e9
-    bf16_tflops = flops / (bf16_ms * 1e-3) / 1e12
-    tr = traffic_per_launch()
     probe = fp8_gemm_probe(dev)
-    cpu = None
-    if not args.no_cpu_baseline:
-        cpu = cpu_baseline(w, g)
-    line = {
-        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 (fp32 accumulate)",
-        "data": "synthetic (seeded, FLUX-style token mix; see fqa_synth)",
-        "config": {"workload": w.name, "B": B, "H": H, "N": N, "d": d,
-                   "n_text": w.n_text, "n_ctx": w.n_ctx, "n_img": w.n_img,
-                   "step": "fqa_quantize + fqa_attention_fp8",
-                   "l2": "inputs larger than L2 (BF16 Q,K,V = %.0f MB per step)" % (3 * 2 * B * H * N * d / 1e6),
-                   "parallelism": f"dp{world} (independent batches)"},
-        "roofline": {"bound": "tensor", "kernel": "attn_fp8_kernel", "achieved": attn_tflops,
-                     "peak": fp8_peak, "unit": "TFLOP/s", "frac": attn_tflops / fp8_peak,
-                     "peak_source": f"{pk_kind}: 2 x bf16_tflops (burst) of MEASURED_PEAKS.json",
-                     "frac_of_nominal_4500": attn_tflops / NOMINAL_FP8_TFLOPS,
-                     "ms_per_launch": attn_ms, "traffic": tr},
-        "quantizer": {"ms": quant_ms, "gbs": quant_gbs, "algorithmic_bytes": quant_bytes,
-                      "frac_of_hbm": quant_gbs / pk["hbm_gbs"], "hbm_peak_gbs": pk["hbm_gbs"]},
-        "bf16_path": {"ms": bf16_ms, "tflops": bf16_tflops, "frac_of_bf16_peak": bf16_tflops / bf16_peak,
-                      "frac_of_nominal_2250": bf16_tflops / NOMINAL_BF16_TFLOPS},
-        "e2e": {"value": job_tflops(flops, world, e2e_ms), "unit": "TFLOP/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-                "pipeline": "two device buffer sets; uploads, kernels and downloads on three streams"},
-        # per step: quantize_fused_kernel + attn_fp8_kernel (plus one
-        # 16-byte cudaMemsetAsync of the quantizer's counters)
-        "gpu_launches": 2 * K,
-        "clocks": clk.summary(),
-        "fp8_gemm_probe": probe,
-        "cpu_baseline": cpu,
-    }
+    cpu = None if args.no_cpu_baseline else cpu_baseline(w, g)
+    line = step_line(w, world, K, args.warmup, ms_per_step, attn_ms, quant_ms, bf16_ms, e2e_ms, h2d, d2h,
+                     clk.summary(), probe, cpu, traffic_per_launch(), pk, pk_kind)
     print(json.dumps(line), flush=True)
 
 
