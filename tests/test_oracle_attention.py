@@ -165,8 +165,10 @@ def test_hand_worked_p_rounding_cases(idx):
     assert np.max(np.abs(out - expect)) < 1e-12
 
 
-def test_config0_quantized_close_to_exact():
-    w = s.workload(0)
+def test_small_workload_quantized_close_to_exact():
+    """On tiny_n256 (no outlier channels) the FP8 scheme stays within
+    cos 0.995 of exact attention."""
+    w = s.workload("tiny_n256")
     g = s.generate(w)
     sc = oracle.softmax_scale()
     qz = oracle.quantize(g["q"], g["k"], g["v"])
