@@ -136,17 +136,20 @@ FQA_API fqa_status fqa_quantize(const void* q, const void* k, const void* v, int
  * convenience.)
  *
  * Same arguments, results and bit-exactness as fqa_quantize(), minus
- * workspace/workspace_bytes.  The K-mean scratch is a fixed array of
- * fqa_quantize_noalloc_max_workspace_bytes() = 8 MiB inside the library, one
- * per GPU that loads it, held until the process exits.  Sizes whose scratch
- * need, fqa_quantize_workspace_bytes(B,H,N,d), exceeds that limit are rejected
- * with FQA_ERR_UNSUPPORTED before anything is launched.  Neither this call nor
+ * workspace/workspace_bytes.  The scratch is a fixed array of
+ * fqa_quantize_noalloc_max_workspace_bytes() = 8 MiB + 256 bytes inside the
+ * library (8 MiB of K-mean partial sums, enough for B*H*ceil(N/64) <= 16384
+ * blocks, plus the launch's counters), one per GPU that loads it, held until
+ * the process exits.  Sizes whose scratch need,
+ * fqa_quantize_workspace_bytes(B,H,N,d), exceeds that limit are rejected with
+ * FQA_ERR_UNSUPPORTED before anything is launched.  Neither this call nor
  * its set-up allocates device memory (no cudaMalloc, cudaFree or allocating
  * library routine).
  *
  * The first call on a device looks up the device address of that device's
- * array (once per device, with that device current); make that first call
- * before any stream capture.  Every call on a device shares the one array and
+ * array (with that device current); make that first call before any stream
+ * capture.  The address is cached only once the lookup succeeds, so a first
+ * call that failed is retried by the next one.  Every call on a device shares the one array and
  * leaves its last contents there; nothing in it needs to start at zero.  Calls
  * that overlap on the GPU (e.g. on two streams at once) race on the array:
  * order them on one stream or synchronize between them.
@@ -156,7 +159,7 @@ FQA_API fqa_status fqa_quantize_noalloc(const void* q, const void* k, const void
                                         float* sk, float* sv, float* sv_max, float* k_mean,
                                         void* cuda_stream);
 
-/* Size of the fixed scratch array fqa_quantize_noalloc() uses (8 MiB). */
+/* Size of the fixed scratch array fqa_quantize_noalloc() uses (8 MiB + 256 bytes). */
 FQA_API size_t fqa_quantize_noalloc_max_workspace_bytes(void);
 
 /*

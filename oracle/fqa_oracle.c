@@ -133,15 +133,23 @@ void orc_k_mean(const uint16_t *k, int B, int H, int N, int d, float *mu)
             }
 }
 
-/* One 64-token block of one head: absmax scale onto 448 and E4M3 codes.
- * x[n*d + c] are the binary32 values to quantize.  Readings: s = amax/448 and
- * inv = 448/amax as binary32 divisions; amax == 0 gives s = inv = 0; the
- * code is E4M3_RNE_sat(fl32(x * inv)) -- the product is rounded to binary32
- * first, then encoded. */
-static void quantize_block(const float *x, int d, uint8_t *codes, float *scale)
+/* One block of one head (n_tok tokens, at most 64): absmax scale onto 448
+ * and E4M3 codes.  x[n*d + c] are the binary32 values to quantize.
+ * Readings: s = amax/448 and inv = 448/amax as binary32 divisions; amax == 0
+ * gives s = inv = 0; the code is E4M3_RNE_sat(fl32(x * inv)) -- the product
+ * is rounded to binary32 first, then encoded.
+ * Two regimes of tiny blocks, on which the pages are silent:
+ *  - 448/amax overflows binary32 (amax below about 1.3e-36; BF16 inputs can
+ *    hold such values): inv = +inf would turn the block's zeros into
+ *    0 * inf = NaN.  The reading keeps the intent, amax onto 448, by dividing
+ *    instead: code = E4M3_RNE_sat(fl32(x / s)).
+ *  - amax / 448 underflows to s = 0 (amax below about 3e-43; only smoothed K,
+ *    whose binary32 differences can be subnormal, gets there): the block is
+ *    flushed, inv = 0, so every code is a signed zero, as for amax == 0. */
+static void quantize_block(const float *x, int n_tok, int d, uint8_t *codes, float *scale)
 {
     float amax = 0.0f;
-    for (int i = 0; i < 64 * d; i++) {
+    for (int i = 0; i < n_tok * d; i++) {
         float a = fabsf(x[i]);
         if (a > amax) amax = a;
     }
@@ -149,9 +157,12 @@ static void quantize_block(const float *x, int d, uint8_t *codes, float *scale)
     if (amax > 0.0f) {
         s = amax / 448.0f;
         inv = 448.0f / amax;
+        if (s == 0.0f)
+            inv = 0.0f;
     }
-    for (int i = 0; i < 64 * d; i++) {
-        float y = x[i] * inv;
+    int divide = isinf(inv);
+    for (int i = 0; i < n_tok * d; i++) {
+        float y = divide ? x[i] / s : x[i] * inv;
         codes[i] = orc_e4m3_encode((double)y);
     }
     *scale = s;
@@ -179,13 +190,13 @@ void orc_quantize(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                 size_t sidx = ((size_t)b * H + h) * nblk + j;
                 for (int i = 0; i < 64 * d; i++)
                     x[i] = orc_bf16_to_float(q[base + i]);
-                quantize_block(x, d, q8 + base, &sq[sidx]);
+                quantize_block(x, 64, d, q8 + base, &sq[sidx]);
                 for (int i = 0; i < 64 * d; i++)
                     x[i] = orc_bf16_to_float(k[base + i]) - mu[i % d];
-                quantize_block(x, d, k8 + base, &sk[sidx]);
+                quantize_block(x, 64, d, k8 + base, &sk[sidx]);
                 for (int i = 0; i < 64 * d; i++)
                     x[i] = orc_bf16_to_float(v[base + i]);
-                quantize_block(x, d, v8 + base, &sv[sidx]);
+                quantize_block(x, 64, d, v8 + base, &sv[sidx]);
                 if (sv[sidx] > vmax) vmax = sv[sidx];
             }
             sv_max[(size_t)b * H + h] = vmax;

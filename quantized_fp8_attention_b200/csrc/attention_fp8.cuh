@@ -44,16 +44,6 @@
 
 namespace fqa {
 
-#ifndef FQA_PINGPONG
-#define FQA_PINGPONG 0
-#endif
-// 1: the two Q tiles' warpgroups take turns for their exponential loops.
-// Off by default: with four softmax warps per sub-partition the MUFU units
-// stay busier when all of them run freely (737 us against 830 us on the
-// 8704-token, 24-head workload).
-constexpr bool kPingPong = FQA_PINGPONG != 0;
-
-
 constexpr int kF8Threads = 640;
 // warp indices: Q/K producer, MMA issuer of tile 0 (and TMEM owner), V
 // producer, MMA issuer of tile 1
@@ -71,8 +61,8 @@ struct F8Traits {
   static constexpr int kOffL = kOffP + 4 * kTileBytes;          // [item parity][tile][half][row]
   static constexpr int kOffBar = kOffL + 2 * 2 * 2 * 128 * 4;
   // fullK, fullV, emptyK, emptyV [kStages]; barQ, barQfree; barS, barSfree,
-  // barP, barPV, barTurn, barDrain, barL [2 each]
-  static constexpr int kNumBars = 4 * kStages + 2 + 14;
+  // barP, barPV, barDrain, barL [2 each]
+  static constexpr int kNumBars = 4 * kStages + 2 + 12;
   static constexpr int kSmemBytes = kOffBar + 8 * kNumBars + 16 + 1024;
 };
 
@@ -132,9 +122,8 @@ __global__ void __launch_bounds__(kF8Threads, 1)
   uint64_t* barSfree = barQ + 4;   // [2] S_t read by its warpgroup
   uint64_t* barP = barQ + 6;       // [2] P_t in shared memory, O_t rescaled
   uint64_t* barPV = barQ + 8;      // [2] PV_t complete
-  uint64_t* barTurn = barQ + 10;   // [2] exponential-loop turns
-  uint64_t* barDrain = barQ + 12;  // [2] error path: an issuer's MMAs completed
-  uint64_t* barL = barQ + 14;      // [2] both halves' row sums written
+  uint64_t* barDrain = barQ + 10;  // [2] error path: an issuer's MMAs completed
+  uint64_t* barL = barQ + 12;      // [2] both halves' row sums written
   float* sL = reinterpret_cast<float*>(smem + T::kOffL);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + T::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -164,7 +153,6 @@ __global__ void __launch_bounds__(kF8Threads, 1)
       mbar_init(&barSfree[t], 2 * kBlockM);
       mbar_init(&barP[t], 2 * kBlockM);
       mbar_init(&barPV[t], 1);
-      mbar_init(&barTurn[t], 2 * kBlockM);
       mbar_init(&barL[t], 2 * kBlockM);
     }
     *abort_flag = 0;
@@ -356,11 +344,6 @@ __global__ void __launch_bounds__(kF8Threads, 1)
         const float alpha = ex2_approx(m - m_new);
         const float2 nm2 = make_float2(-m_new, -m_new);
         const float2 a2 = make_float2(ah, ah);
-        if (kPingPong && (t == 1 || g > 0)) {
-          // turn k of tile 1 follows turn k of tile 0
-          const uint32_t par = (t == 0) ? ((g - 1) & 1) : (g & 1);
-          if (!(ok = __all_sync(0xffffffffu, mbar_wait(&barTurn[t], par, abort_flag, p.status)))) break;
-        }
         float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
         const uint32_t pbuf = prow + (uint32_t)(g & 1) * T::kTileBytes;
         const float2 c2 = make_float2(cpv, cpv);
@@ -395,7 +378,6 @@ __global__ void __launch_bounds__(kF8Threads, 1)
           st_shared_v4(pbuf + ((c0 ^ sw) << 4), pw[0], pw[1], pw[2], pw[3]);
           st_shared_v4(pbuf + (((c0 + 1) ^ sw) << 4), pw[4], pw[5], pw[6], pw[7]);
         }
-        if (kPingPong) mbar_arrive(&barTurn[t ^ 1]);   // hand the turn to the other tile
         const float2 l2 = f2_add(ls[0], ls[1]);
         if (j > 0) {
           // O_t holds PV_t(g-1) once it completed; rescale this half's

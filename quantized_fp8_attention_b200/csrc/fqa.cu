@@ -22,11 +22,12 @@ __device__ uint32_t g_status_word;
 
 constexpr int kMaxDevices = 64;
 
+// Per-device lookups, cached only once they succeed: a failed first call
+// (e.g. one made while a stream is being captured) is retried by the next.
 struct DeviceCache {
-  std::once_flag once;
+  std::mutex mu;
   uint32_t* status = nullptr;
   int num_sms = 0;
-  cudaError_t err = cudaSuccess;
 };
 DeviceCache g_dev[kMaxDevices];
 
@@ -44,16 +45,18 @@ static uint32_t* status_ptr(fqa_status* st) {
     return nullptr;
   }
   DeviceCache& c = g_dev[dev];
-  std::call_once(c.once, [&c, dev]() {
+  std::lock_guard<std::mutex> lock(c.mu);
+  if (c.status == nullptr) {
     void* p = nullptr;
-    c.err = cudaGetSymbolAddress(&p, g_status_word);
-    if (c.err == cudaSuccess) c.status = static_cast<uint32_t*>(p);
-    if (c.err == cudaSuccess)
-      c.err = cudaDeviceGetAttribute(&c.num_sms, cudaDevAttrMultiProcessorCount, dev);
-  });
-  if (c.err != cudaSuccess || c.status == nullptr) {
-    *st = FQA_ERR_CUDA;
-    return nullptr;
+    int sms = 0;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        p == nullptr || sms <= 0) {
+      *st = FQA_ERR_CUDA;
+      return nullptr;
+    }
+    c.num_sms = sms;
+    c.status = static_cast<uint32_t*>(p);
   }
   return c.status;
 }
@@ -103,9 +106,11 @@ static fqa_status launch_status() {
   return cudaGetLastError() == cudaSuccess ? FQA_OK : FQA_ERR_CUDA;
 }
 
+// SM count of the current device (valid once status_ptr() succeeded on it).
 static int num_sms() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  std::lock_guard<std::mutex> lock(g_dev[dev].mu);
   return g_dev[dev].num_sms;
 }
 
@@ -316,9 +321,11 @@ fqa_status fqa_debug_status(void* cuda_stream, uint32_t* flags_out) {
 // the library instead of a caller-provided workspace.
 namespace fqa {
 
-// Upper bound of the scratch the quantizer needs, B*H*(N/64)*128*4 bytes:
-// 8 MiB covers B*H*(N/64) <= 16384 (e.g. B=2, H=24, N=16896 needs 6.2 MiB).
-constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;
+// The scratch fqa_quantize needs is the K-mean partial sums,
+// B*H*ceil(N/64)*128*4 bytes rounded up to 256, plus 256 bytes of counters.
+// 8 MiB of partial sums covers B*H*ceil(N/64) <= 16384 blocks (B=2, H=24,
+// N=16896 needs 6.2 MiB); the array holds that plus the counters.
+constexpr size_t kNoAllocScratchBytes = (size_t(8) << 20) + 256;
 
 // One copy per GPU that loads the library, held until the process exits.
 // In host code this name is only a stand-in: the device address comes from
@@ -326,14 +333,14 @@ constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;
 static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
 
 struct NoAllocCache {
-  std::once_flag once;
+  std::mutex mu;
   float* ptr = nullptr;
-  cudaError_t err = cudaSuccess;
 };
 NoAllocCache g_noalloc[kMaxDevices];
 
-// Device address of this device's scratch array, looked up once per device
-// with that device current.
+// Device address of this device's scratch array, looked up with that device
+// current; cached once the lookup succeeds (a failed lookup, e.g. during a
+// stream capture, is retried by the next call).
 static float* noalloc_scratch(fqa_status* st) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
@@ -341,14 +348,14 @@ static float* noalloc_scratch(fqa_status* st) {
     return nullptr;
   }
   NoAllocCache& c = g_noalloc[dev];
-  std::call_once(c.once, [&c]() {
+  std::lock_guard<std::mutex> lock(c.mu);
+  if (c.ptr == nullptr) {
     void* p = nullptr;
-    c.err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (c.err == cudaSuccess) c.ptr = static_cast<float*>(p);
-  });
-  if (c.err != cudaSuccess || c.ptr == nullptr) {
-    *st = FQA_ERR_CUDA;
-    return nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      *st = FQA_ERR_CUDA;
+      return nullptr;
+    }
+    c.ptr = static_cast<float*>(p);
   }
   return c.ptr;
 }

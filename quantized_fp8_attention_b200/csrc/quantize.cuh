@@ -39,18 +39,12 @@ namespace fqa {
 // units in flight.  Thread t handles the 16-byte chunks t, t+T, t+2T, ... of
 // a unit (T threads, 8 channels a chunk).  Every wait is bounded.
 
-#ifndef FQA_QUANT_THREADS
-#define FQA_QUANT_THREADS 256
-#endif
-#ifndef FQA_QUANT_RING_KB
-#define FQA_QUANT_RING_KB 64
-#endif
-constexpr int kQuantThreads = FQA_QUANT_THREADS;
+constexpr int kQuantThreads = 256;
 constexpr int kQuantWarps = kQuantThreads / 32;
 constexpr int kBlockBytes = kQBlock * kHeadDim * 2;            // 16 KB of BF16
 constexpr int kChunks = kBlockBytes / 16 / kQuantThreads;       // 16-byte chunks per thread
 constexpr int kVals = 8 * kChunks;
-constexpr int kRingBytes = FQA_QUANT_RING_KB * 1024;
+constexpr int kRingBytes = 64 * 1024;             // three CTAs per SM
 constexpr int kMaxSlots = kRingBytes / kBlockBytes;
 constexpr int kQuantSmem = kRingBytes + 128;
 constexpr int kPartialRowsPerSlot = kBlockBytes / (kHeadDim * 4);   // 32 partial rows per 16 KB
@@ -126,7 +120,21 @@ __device__ __forceinline__ float quantize_chunks(float (&x)[kVals], float* red, 
 #pragma unroll
   for (int w = 1; w < kQuantWarps; ++w) a = fmaxf(a, red[slot * kQuantWarps + w]);
   const float scale = a > 0.0f ? __fdiv_rn(a, 448.0f) : 0.0f;
-  const float inv = a > 0.0f ? __fdiv_rn(448.0f, a) : 0.0f;
+  float inv = a > 0.0f ? __fdiv_rn(448.0f, a) : 0.0f;
+  if (scale == 0.0f) inv = 0.0f;               // amax / 448 underflowed: flush the block
+  if (isinf(inv)) {
+    // 448 / amax overflowed (amax below about 1.3e-36): codes of x / scale,
+    // so the block's zeros stay zeros instead of 0 * inf.  Block-uniform.
+#pragma unroll
+    for (int i = 0; i < kChunks; ++i) {
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        w[e] = e4m3x2(__fdiv_rn(x[8 * i + 2 * e], scale), __fdiv_rn(x[8 * i + 2 * e + 1], scale));
+      st_global_v2_hint(dst + 8 * (t + kQuantThreads * i), w[0] | (w[1] << 16), w[2] | (w[3] << 16), policy);
+    }
+    return scale;
+  }
 #pragma unroll
   for (int i = 0; i < kChunks; ++i) {
     uint32_t lo = e4m3x2(__fmul_rn(x[8 * i], inv), __fmul_rn(x[8 * i + 1], inv));

@@ -22,7 +22,9 @@ int main(void) {
   /* B*H*(N/64)*d*4 rounded up to 256, plus 256 bytes of counters */
   CHECK(fqa_quantize_workspace_bytes(1, 24, 8704, 128) == 1671168 + 256);
   CHECK(fqa_quantize_workspace_bytes(1, 1, 100, 128) == 0);
-  CHECK(fqa_quantize_noalloc_max_workspace_bytes() == (size_t)8 << 20);
+  /* 8 MiB of partial sums plus the 256 counter bytes: exactly 16384 blocks fit */
+  CHECK(fqa_quantize_noalloc_max_workspace_bytes() == ((size_t)8 << 20) + 256);
+  CHECK(fqa_quantize_workspace_bytes(1, 16, 65536, 128) == fqa_quantize_noalloc_max_workspace_bytes());
   /* argument errors come back before anything is launched */
   void* p = (void*)(uintptr_t)0x10000;
   float* f = (float*)p;

@@ -83,13 +83,14 @@ def test_fp8_attention_matches_oracle(idx):
     ex = oracle.attention_exact(g["q"], g["k"], g["v"], U.SCALE, heads=heads, rows=rows)
     cos_gpu = U.metrics(got32, ex)["cos"]
     cos_orc = U.metrics(ref, ex)["cos"]
-    print(f"[{w.name}] cos vs exact FP64: gpu {cos_gpu:.6f}  oracle {cos_orc:.6f}")
+    print(f"[{w.name}] cos vs exact FP64: gpu {cos_gpu:.6f}  oracle {cos_orc:.6f}  "
+          f"meets 0.995: {cos_gpu >= 0.995}")
     assert cos_gpu >= cos_orc - 1e-3
     if cos_orc >= 0.995:
         assert cos_gpu >= 0.995
 
 
-@pytest.mark.parametrize("idx", [0, 1, 3])
+@pytest.mark.parametrize("idx", [0, 1, 2, 3, 4])
 def test_bf16_attention_matches_exact(idx):
     fqa = _fqa()
     w = synth.workload(idx)
@@ -108,6 +109,29 @@ def test_bf16_attention_matches_exact(idx):
     assert np.all(np.abs(got - ex) <= 2e-2 + 2.0 ** -8 * np.abs(ex))
     b16 = out16.view(torch.int16).cpu().numpy().view(np.uint16)
     assert np.array_equal(b16, oracle.bf16_round(out32.cpu().numpy().astype(np.float64)))
+
+
+# The scheme's own ceiling (the oracle's cos against exact FP64) is below 0.995
+# on the four workloads with x20 outlier channels; these cases stay visible as
+# expected failures instead of being dropped.
+_CEILING = "scheme ceiling: the oracle itself stays below cos 0.995 on x20 outlier channels"
+
+
+@pytest.mark.parametrize("idx", [0] + [pytest.param(i, marks=pytest.mark.xfail(reason=_CEILING, strict=True))
+                                       for i in (1, 2, 3, 4)])
+def test_fp8_cos_target_vs_exact(idx):
+    """The accuracy target: cos >= 0.995 against exact unquantized FP64
+    attention (sampled heads x rows on the large workloads)."""
+    fqa = _fqa()
+    w = synth.workload(idx)
+    g = U.host_inputs(idx)
+    q, k, v = (U.to_device(g[t]) for t in "qkv")
+    out32 = fqa.attention_fp8(fqa.quantize(q, k, v), U.SCALE, fqa.FQA_OUT_F32)
+    heads, rows = _rows_heads(w)
+    ex = oracle.attention_exact(g["q"], g["k"], g["v"], U.SCALE, heads=heads, rows=rows)
+    cos = U.metrics(_pick(out32.cpu().numpy(), heads, rows), ex)["cos"]
+    print(f"\n[{w.name}] FP8 cos vs exact FP64: {cos:.6f} (target 0.995)")
+    assert cos >= 0.995
 
 
 def _gen(shape, seed, scale=1.0):

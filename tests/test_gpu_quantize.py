@@ -121,3 +121,28 @@ def test_bounded_wait_times_out_and_context_survives():
     got = U.to_oracle_quant(fqa.quantize(q, k, v))
     ref = U.oracle_quant(0)
     assert np.array_equal(got["q8"], ref["q8"])
+
+
+def test_quantize_tiny_blocks():
+    """Blocks whose 448/amax overflows binary32 (codes from x / s) and a
+    smoothed-K block whose scale underflows (flushed to signed zeros):
+    bit-exact against the oracle, and no NaN code (S.1111.111) anywhere."""
+    fqa = _fqa()
+    N = 1024
+    x = np.zeros((1, 2, N, 128))
+    x[0, 0, 0, 0] = 2.0 ** -123
+    x[0, 0, 1, 5] = -(2.0 ** -123)
+    x[0, 0, 2, 9] = 2.0 ** -130
+    x[0, 0, 3, 127] = 2.0 ** -133
+    x[0, 1, 1000, 0] = 2.0 ** -133          # head 1: K mean 2^-143, blocks 0..14 flushed
+    x[0, 0, 64:128] = np.random.default_rng(12).standard_normal((64, 128))   # an ordinary block
+    bits = synth.round_to_bf16_bits(x)
+    ref = oracle.quantize(bits, bits, bits)
+    t = U.to_device(bits)
+    got = U.to_oracle_quant(fqa.quantize(t, t, t))
+    torch.cuda.synchronize()
+    for name in ref:
+        assert np.array_equal(np.asarray(got[name]).view(np.uint8), np.asarray(ref[name]).view(np.uint8)), name
+    for name in ("q8", "k8", "v8"):
+        assert not np.any((got[name] & 0x7F) == 0x7F), name
+    assert fqa.fqa_debug_status()[0] == fqa.FQA_OK

@@ -125,3 +125,80 @@ def test_k_smoothing_absorbs_channel_offset():
     b = oracle.quantize(_bf16(k), _bf16(k + off), _bf16(k))
     assert np.array_equal(a["k8"], b["k8"]) and np.array_equal(a["sk"], b["sk"])
     assert np.array_equal(b["k_mean"] - a["k_mean"], off[None, None, :].astype(np.float32))
+
+
+# ---------------------------------------------------------------- tiny blocks
+# Two regimes where the plain rule code = E4M3(fl32(x * fl32(448/amax))) has
+# no finite answer; the pages are silent on both, so the readings are:
+#   448/amax overflows binary32  -> code = E4M3(fl32(x / s)), s = fl32(amax/448)
+#   amax/448 underflows to s = 0 -> the block is flushed: inv = 0, signed-zero codes
+# The expected values below were worked by hand; the comments give the steps.
+
+def _bits(x: float) -> int:
+    """BF16 bit pattern of a value exactly representable in BF16."""
+    b = s.round_to_bf16_bits(np.array([x], dtype=np.float64))[0]
+    assert s.bf16_bits_to_f32(np.array([b], np.uint16))[0] == np.float32(x)
+    return int(b)
+
+
+def test_block_whose_inverse_scale_overflows_divides_by_the_scale():
+    # amax = 2^-123 (a BF16 normal); 448 * 2^123 = 7 * 2^129 > FLT_MAX, so
+    # inv overflows.  s = fl32(2^-123 / 448) = fl32(2^-129 / 7): subnormal,
+    # 2^20 / 7 = 149796.57 units of 2^-149 -> 149797 * 2^-149.
+    #   x =  2^-123: x/s = 2^26/149797 = 447.998 -> 448       -> 0x7E
+    #   x = -2^-123:                              -> -448     -> 0xFE
+    #   x =  2^-130 (BF16 subnormal): 2^19/149797 = 3.49999 -> 3.5 = 1.75*2^1 -> 0x46
+    #   x =  2^-133 (smallest BF16): 2^16/149797 = 0.437505 -> 0.4375 = 1.75*2^-2 -> 0x2E
+    #   x =  0                                               -> 0x00 (not 0*inf = NaN)
+    blk = np.zeros((1, 1, 64, 128), dtype=np.uint16)
+    blk[0, 0, 0, 0] = _bits(2.0 ** -123)
+    blk[0, 0, 1, 5] = _bits(-(2.0 ** -123))
+    blk[0, 0, 2, 9] = _bits(2.0 ** -130)
+    blk[0, 0, 3, 127] = _bits(2.0 ** -133)
+    z = np.zeros_like(blk)
+    r = oracle.quantize(blk, z, blk)
+    s_expect = np.float32(149797 * 2.0 ** -149)
+    assert r["sq"][0, 0, 0] == s_expect and r["sv"][0, 0, 0] == s_expect
+    assert r["sv_max"][0, 0] == s_expect
+    for name in ("q8", "v8"):
+        c = r[name][0, 0]
+        assert (c[0, 0], c[1, 5], c[2, 9], c[3, 127]) == (0x7E, 0xFE, 0x46, 0x2E)
+        nz = np.zeros_like(c, dtype=bool)
+        nz[0, 0] = nz[1, 5] = nz[2, 9] = nz[3, 127] = True
+        assert np.all(c[~nz] == 0)                    # zeros stay zeros
+    # the same numbers from exact rational arithmetic and the spec's code table
+    from fractions import Fraction as F
+    table = {i: oracle.e4m3_decode(i) for i in range(256) if not np.isnan(oracle.e4m3_decode(i))}
+    sF = F(149797, 2 ** 149)
+    for x, code in ((F(1, 2 ** 123), 0x7E), (F(1, 2 ** 130), 0x46), (F(1, 2 ** 133), 0x2E)):
+        y = float(np.float32(float(x / sF)))          # the binary32 quotient
+        best = min((c for c in table if table[c] >= 0), key=lambda c: abs(table[c] - y))
+        assert best == code
+
+
+def test_smoothed_k_block_whose_scale_underflows_is_flushed():
+    # N = 1024, channel 0 of K holds 2^-133 at token 1000 and 0 elsewhere:
+    #   mu[0] = 2^-133 / 1024 = 2^-143 (exact: 64 units of 2^-149)
+    #   blocks 0..14: x = 0 - 2^-143 in channel 0, 0 elsewhere; amax = 2^-143,
+    #     s = fl32(2^-143 / 448) = fl32(0.1429 * 2^-149) = 0  -> flushed: s = 0,
+    #     codes fl32(x * 0) = -0 -> 0x80 in channel 0, +0 -> 0x00 elsewhere
+    #   block 15 (tokens 960..1023): x(token 1000) = 2^-133 - 2^-143 =
+    #     65472 * 2^-149 = amax; s = fl32(65472/448 = 146.14 units) = 146 * 2^-149;
+    #     448/amax overflows -> divide: 65472/146 = 448.4 -> 0x7E;
+    #     the other tokens: -64/146 = -0.4384 -> -0.4375 -> 0xAE
+    N = 1024
+    k = np.zeros((1, 1, N, 128), dtype=np.uint16)
+    k[0, 0, 1000, 0] = _bits(2.0 ** -133)
+    z = np.zeros_like(k)
+    r = oracle.quantize(z, k, z)
+    assert r["k_mean"][0, 0, 0] == np.float32(2.0 ** -143) and np.all(r["k_mean"][0, 0, 1:] == 0)
+    sk, k8 = r["sk"][0, 0], r["k8"][0, 0]
+    assert np.all(sk[:15] == 0) and sk[15] == np.float32(146 * 2.0 ** -149)
+    assert np.all(k8[:960, 0] == 0x80) and np.all(k8[:960, 1:] == 0x00)
+    assert k8[1000, 0] == 0x7E
+    other = np.ones(64, dtype=bool)
+    other[40] = False
+    assert np.all(k8[960:][other, 0] == 0xAE) and np.all(k8[960:, 1:] == 0x00)
+    # no code anywhere is a NaN (S.1111.111)
+    for name in ("q8", "k8", "v8"):
+        assert not np.any((r[name] & 0x7F) == 0x7F)

@@ -2,8 +2,8 @@
 
 fqa_quantize_noalloc serves callers that cannot allocate device memory at
 call time (for example an operator inside a host framework that owns all
-device memory): it keeps the K-mean scratch in a fixed 8 MiB array inside the
-library instead of taking a workspace.  Its results must equal those of the
+device memory): it keeps the K-mean scratch and its counters in a fixed array
+(8 MiB + 256 bytes) inside the library instead of taking a workspace.  Its results must equal those of the
 workspace entry point bit for bit (the quantizer's tolerance), on two calls in
 a row -- the second on a different workload, so stale scratch contents from
 the first call cannot leak into it.  This file is collected last on purpose.
@@ -28,7 +28,9 @@ def test_noalloc_matches_workspace_entry_point_twice():
     import quantized_fp8_attention_b200 as fqa
     L = fqa.lib()
     L.fqa_quantize_noalloc_max_workspace_bytes.restype = ctypes.c_size_t
-    assert L.fqa_quantize_noalloc_max_workspace_bytes() == 8 << 20
+    assert L.fqa_quantize_noalloc_max_workspace_bytes() == (8 << 20) + 256
+    # exactly 16384 blocks of partial sums fit (1 x 16 heads x 65536 tokens)
+    assert fqa.fqa_quantize_workspace_bytes(1, 16, 65536) == (8 << 20) + 256
     for idx in (3, 1):                       # two calls in a row, different sizes
         g = U.host_inputs(idx)
         q, k, v = (U.to_device(g[t]) for t in "qkv")
@@ -48,7 +50,7 @@ def test_noalloc_matches_workspace_entry_point_twice():
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
     import quantized_fp8_attention_b200 as fqa
-    # B*H*(N/64)*128*4 bytes = 1*48*1024*512 = 24 MiB > 8 MiB: refused with
+    # B*H*(N/64)*128*4 bytes = 1*48*1024*512 = 24 MiB > 8 MiB + 256: refused with
     # FQA_ERR_UNSUPPORTED before anything is launched (the pointers below are
     # never dereferenced)
     P = ctypes.c_void_p
