@@ -36,8 +36,10 @@
  *    NULL = the legacy default stream).  No call synchronizes, except
  *    fqa_debug_status().
  *  - Layouts are row-major and contiguous: [B, H, N, d] with d innermost.
- *  - v1 limits: d == 128; N a multiple of 128 (quantizer: of 64);
- *    1 <= N <= 65536; B, H >= 1, B*H <= 65535, B*H*N < 2^31; device pointers
+ *  - Limits: d == 128; any 1 <= N <= 65536 (real prompt lengths: the last
+ *    64-token block and the last 128-key tile of a head may be short; see
+ *    fqa_quantize and fqa_attention_fp8); B, H >= 1, B*H <= 65535,
+ *    B*H*N < 2^31; device pointers
  *    16-byte aligned (the block-scale arrays and sv_max 4-byte aligned; k_mean
  *    16-byte aligned); a finite softmax_scale > 0; outputs must not overlap
  *    inputs.
@@ -68,7 +70,7 @@ extern "C" {
 typedef enum {
   FQA_OK = 0,
   FQA_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, bad dtype, small workspace */
-  FQA_ERR_UNSUPPORTED = 2,  /* d != 128, N not a multiple of 128 (64), sizes beyond the limits */
+  FQA_ERR_UNSUPPORTED = 2,  /* d != 128, sizes beyond the limits */
   FQA_ERR_MISALIGNED = 3,   /* a pointer not aligned as required */
   FQA_ERR_CUDA = 4,         /* a CUDA runtime / driver call or launch failed */
   FQA_ERR_TIMEOUT = 5       /* a bounded device wait gave up (from fqa_debug_status) */
@@ -86,8 +88,8 @@ FQA_API int fqa_version(void);
 FQA_API const char* fqa_status_string(fqa_status status);
 
 /*
- * Bytes of device workspace fqa_quantize() needs: B*H*(N/64)*d*4 rounded up
- * to a multiple of 256 (the per-64-token-block partial sums of the K mean),
+ * Bytes of device workspace fqa_quantize() needs: B*H*ceil(N/64)*d*4 rounded
+ * up to a multiple of 256 (the per-64-token-block partial sums of the K mean),
  * plus 256 (the launch's grid-barrier and work-queue counters).  Returns 0
  * for invalid sizes.
  */
@@ -97,22 +99,26 @@ FQA_API size_t fqa_quantize_workspace_bytes(int B, int H, int N, int d);
  * fqa_quantize -- BF16 Q, K, V -> E4M3 codes and FP32 block scales.
  * [RTX-DE] SDPA quantization paragraph: Q, K and V are the quantized inputs.
  *
- * For each (b, h):
- *   k_mean[c] = (sum over 64-token blocks j, ascending, of the sequential
- *               binary32 sum of K over the block's 64 tokens) / N
+ * For each (b, h), with blocks of 64 tokens (the last one holds the
+ * N - 64*(ceil(N/64)-1) remaining tokens):
+ *   k_mean[c] = (sum over blocks j, ascending, of the sequential binary32 sum
+ *               of K over the block's tokens) / N
  *               (pinned order, one round-to-nearest division);
- *   for each 64-token block and tensor X in {Q, K - k_mean, V} (the K
- *   difference is one binary32 subtraction per element):
- *     amax = max |X| over the 64 x 128 block;
+ *   for each block and tensor X in {Q, K - k_mean, V} (the K difference is
+ *   one binary32 subtraction per element):
+ *     amax = max |X| over the block's tokens x 128 channels;
  *     scale = amax / 448, inv = 448 / amax (binary32 divisions; both 0 if amax = 0);
  *     code  = E4M3 round-to-nearest-even, saturating, of fl32(X * inv);
+ *     tiny blocks: where inv overflows binary32 the code is that of
+ *     fl32(X / scale), and where scale underflows to 0 the block is flushed
+ *     (inv = 0, signed-zero codes) -- finite inputs never give NaN codes;
  *   sv_max = max over blocks of the V scales.
  * The results are bit-exact functions of the inputs (no atomics that change
  * values, no order dependence).
  *
  * q, k, v      in : BF16 [B,H,N,d]
  * q8, k8, v8   out: E4M3 codes, uint8 [B,H,N,d] (same layout as the inputs)
- * sq, sk, sv   out: FP32 [B,H,N/64] block scales
+ * sq, sk, sv   out: FP32 [B,H,ceil(N/64)] block scales
  * sv_max       out: FP32 [B,H]
  * k_mean       out: FP32 [B,H,d]
  * workspace    scratch of at least fqa_quantize_workspace_bytes(B,H,N,d)
@@ -178,6 +184,10 @@ FQA_API size_t fqa_quantize_noalloc_max_workspace_bytes(void);
  * Evaluated in binary32: x = fl(S * a) rounded toward zero, then x - m, so
  * the row maximum gets p = 1 exactly; a P code whose binary32 value lies
  * within evaluation error of an E4M3 rounding midpoint may round either way.
+ * Any N: the last tile holds the N % 128 remaining keys (when nonzero) and
+ * keys past N take no part (no maximum, row-sum term or P code); the row
+ * sum's correction for them is a binary32 subtraction, so l may differ from
+ * a sum that never had them by a few ulp.
  * Enqueues one persistent kernel launch (one CTA per SM).
  *
  * out: [B,H,N,d] BF16 (FQA_OUT_BF16) or FP32 (FQA_OUT_F32).
@@ -191,8 +201,8 @@ FQA_API fqa_status fqa_attention_fp8(const void* q8, const void* k8, const void*
 /*
  * fqa_attention_bf16 -- the unquantized comparison path ([KLEIN], VANILLA
  * BF16 attention): softmax(Q K^T * softmax_scale) V with BF16 operands, FP32
- * accumulation and online softmax over 128-key tiles, P rounded to BF16 for
- * the P.V product, out = O / l.
+ * accumulation and online softmax over 128-key tiles (the last one holds the
+ * N % 128 remaining keys), P rounded to BF16 for the P.V product, out = O / l.
  *
  * q, k, v: BF16 [B,H,N,d]; out: [B,H,N,d] BF16 or FP32.
  */

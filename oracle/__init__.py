@@ -128,17 +128,18 @@ def k_mean(k_bf16: np.ndarray) -> np.ndarray:
 
 
 def quantize(q: np.ndarray, k: np.ndarray, v: np.ndarray) -> dict:
-    """BF16 bit arrays [B,H,N,d] -> codes (natural layout) and FP32 scales."""
+    """BF16 bit arrays [B,H,N,d], any N >= 1 -> codes (natural layout) and FP32
+    scales [B,H,ceil(N/64)]."""
     B, H, N, d = q.shape
-    assert N % 64 == 0
+    nb = (N + 63) // 64                    # the last block may be short
     q = np.ascontiguousarray(q, dtype=np.uint16)
     k = np.ascontiguousarray(k, dtype=np.uint16)
     v = np.ascontiguousarray(v, dtype=np.uint16)
     r = dict(
         q8=np.empty((B, H, N, d), np.uint8), k8=np.empty((B, H, N, d), np.uint8),
         v8=np.empty((B, H, N, d), np.uint8),
-        sq=np.empty((B, H, N // 64), np.float32), sk=np.empty((B, H, N // 64), np.float32),
-        sv=np.empty((B, H, N // 64), np.float32), sv_max=np.empty((B, H), np.float32),
+        sq=np.empty((B, H, nb), np.float32), sk=np.empty((B, H, nb), np.float32),
+        sv=np.empty((B, H, nb), np.float32), sv_max=np.empty((B, H), np.float32),
         k_mean=np.empty((B, H, d), np.float32))
     lib().orc_quantize(_p(q), _p(k), _p(v), B, H, N, d, _p(r["q8"]), _p(r["k8"]), _p(r["v8"]),
                        _p(r["sq"]), _p(r["sk"]), _p(r["sv"]), _p(r["sv_max"]), _p(r["k_mean"]))

@@ -113,11 +113,13 @@ uint16_t orc_bf16_round(double x)
 
 /* K per-channel mean, pinned order [reading: the pages give no summation
  * order]: p_j[c] = ((0 + k[64j][c]) + k[64j+1][c]) + ... in binary32 over the
- * 64 tokens of block j; T[c] = ((0 + p_0[c]) + p_1[c]) + ... over blocks;
- * mu[c] = T[c] / (float)N, one binary32 division. */
+ * tokens of block j (64 of them; the last block of a sequence whose length is
+ * not a multiple of 64 holds the remaining N - 64*(nblk-1)); T[c] =
+ * ((0 + p_0[c]) + p_1[c]) + ... over blocks; mu[c] = T[c] / (float)N, one
+ * binary32 division. */
 void orc_k_mean(const uint16_t *k, int B, int H, int N, int d, float *mu)
 {
-    int nblk = N / 64;
+    int nblk = (N + 63) / 64;
     #pragma omp parallel for collapse(2) schedule(static)
     for (int b = 0; b < B; b++)
         for (int h = 0; h < H; h++)
@@ -125,7 +127,8 @@ void orc_k_mean(const uint16_t *k, int B, int H, int N, int d, float *mu)
                 float T = 0.0f;
                 for (int j = 0; j < nblk; j++) {
                     float p = 0.0f;
-                    for (int n = 64 * j; n < 64 * j + 64; n++)
+                    int n1 = 64 * j + 64 < N ? 64 * j + 64 : N;
+                    for (int n = 64 * j; n < n1; n++)
                         p = p + orc_bf16_to_float(k[IDX4(b, h, n, c, H, N, d)]);
                     T = T + p;
                 }
@@ -168,16 +171,18 @@ static void quantize_block(const float *x, int n_tok, int d, uint8_t *codes, flo
     *scale = s;
 }
 
-/* The whole quantizer.  Inputs BF16 [B,H,N,d]; codes written in the same
- * natural [B,H,N,d] layout (the CUDA library's own V layout is its business);
- * sq, sk, sv: [B,H,N/64]; sv_max: [B,H]; k_mean: [B,H,d].
- * K is smoothed as fl32(k - mu[c]) before its block scales are taken. */
+/* The whole quantizer.  Inputs BF16 [B,H,N,d], any N >= 1; codes written in
+ * the same natural [B,H,N,d] layout (the CUDA library's own V layout is its
+ * business); sq, sk, sv: [B,H,ceil(N/64)]; sv_max: [B,H]; k_mean: [B,H,d].
+ * K is smoothed as fl32(k - mu[c]) before its block scales are taken.
+ * [reading] When N is not a multiple of 64 the last block of each head holds
+ * the remaining tokens and its scale is the absmax of those tokens alone. */
 void orc_quantize(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                   int B, int H, int N, int d,
                   uint8_t *q8, uint8_t *k8, uint8_t *v8,
                   float *sq, float *sk, float *sv, float *sv_max, float *k_mean)
 {
-    int nblk = N / 64;
+    int nblk = (N + 63) / 64;
     orc_k_mean(k, B, H, N, d, k_mean);
     #pragma omp parallel for collapse(2) schedule(dynamic)
     for (int b = 0; b < B; b++)
@@ -186,17 +191,18 @@ void orc_quantize(const uint16_t *q, const uint16_t *k, const uint16_t *v,
             const float *mu = k_mean + ((size_t)b * H + h) * d;
             float vmax = 0.0f;
             for (int j = 0; j < nblk; j++) {
+                int nt = N - 64 * j < 64 ? N - 64 * j : 64;
                 size_t base = IDX4(b, h, 64 * j, 0, H, N, d);
                 size_t sidx = ((size_t)b * H + h) * nblk + j;
-                for (int i = 0; i < 64 * d; i++)
+                for (int i = 0; i < nt * d; i++)
                     x[i] = orc_bf16_to_float(q[base + i]);
-                quantize_block(x, 64, d, q8 + base, &sq[sidx]);
-                for (int i = 0; i < 64 * d; i++)
+                quantize_block(x, nt, d, q8 + base, &sq[sidx]);
+                for (int i = 0; i < nt * d; i++)
                     x[i] = orc_bf16_to_float(k[base + i]) - mu[i % d];
-                quantize_block(x, 64, d, k8 + base, &sk[sidx]);
-                for (int i = 0; i < 64 * d; i++)
+                quantize_block(x, nt, d, k8 + base, &sk[sidx]);
+                for (int i = 0; i < nt * d; i++)
                     x[i] = orc_bf16_to_float(v[base + i]);
-                quantize_block(x, 64, d, v8 + base, &sv[sidx]);
+                quantize_block(x, nt, d, v8 + base, &sv[sidx]);
                 if (sv[sidx] > vmax) vmax = sv[sidx];
             }
             sv_max[(size_t)b * H + h] = vmax;
@@ -210,7 +216,9 @@ void orc_quantize(const uint16_t *q, const uint16_t *k, const uint16_t *v,
  * operands: qc [N,d], kc [N,d], vc [N,d] are the code VALUES (not yet
  * multiplied by their block scales), sq/sk/sv the per-64-token scales.
  *
- * For query row i (block I = i/64), KV tiles t of bc keys in ascending order:
+ * For query row i (block I = i/64), KV tiles t of bc keys in ascending order
+ * (when bc does not divide N, the last tile holds the remaining keys; there
+ * are no keys beyond N to mask):
  *   x_ij   = (sum_c qc_ic kc_jc) * sq_I * sk_J * scale * log2(e)
  *   m_t    = max(m_{t-1}, max_{j in t} x_ij),  m_{-1} = -inf  (exact, no
  *            threshold / lazy rescale)
@@ -345,7 +353,7 @@ void orc_attention_fp8(const uint8_t *q8, const uint8_t *k8, const uint8_t *v8,
                        const int *heads, int n_heads, const int *rows, int n_rows,
                        double *out, double *amb, int *namb)
 {
-    int nblk = N / 64;
+    int nblk = (N + 63) / 64;
     (void)B;
     double *qc = (double *)malloc(sizeof(double) * N * d);
     double *kc = (double *)malloc(sizeof(double) * N * d);

@@ -181,8 +181,14 @@ def _require_qkv(q, k, v, dtype: torch.dtype):
     return tuple(q.shape)
 
 
+def nblocks(N: int) -> int:
+    """64-token blocks per head: ceil(N / 64) (the last one may be short)."""
+    return (N + 63) // 64
+
+
 def _require_quantized(qz: "Quantized", B: int, H: int, N: int) -> None:
-    shapes = ((B, H, N, HEAD_DIM),) * 3 + ((B, H, N // 64),) * 3 + ((B, H), (B, H, HEAD_DIM))
+    nb = nblocks(N)
+    shapes = ((B, H, N, HEAD_DIM),) * 3 + ((B, H, nb),) * 3 + ((B, H), (B, H, HEAD_DIM))
     for name, t, shape in zip(Quantized._fields, qz, shapes):
         _require(t, torch.uint8 if name.endswith("8") else torch.float32, name, shape)
 
@@ -191,7 +197,7 @@ class Quantized(NamedTuple):
     q8: torch.Tensor       # uint8 E4M3 codes [B,H,N,128]
     k8: torch.Tensor
     v8: torch.Tensor
-    sq: torch.Tensor       # float32 [B,H,N/64]
+    sq: torch.Tensor       # float32 [B,H,ceil(N/64)]
     sk: torch.Tensor
     sv: torch.Tensor
     sv_max: torch.Tensor   # float32 [B,H]
@@ -201,9 +207,10 @@ class Quantized(NamedTuple):
 def alloc_quantized(B: int, H: int, N: int, device) -> Quantized:
     u8 = dict(dtype=torch.uint8, device=device)
     f32 = dict(dtype=torch.float32, device=device)
+    nb = nblocks(N)
     return Quantized(torch.empty(B, H, N, HEAD_DIM, **u8), torch.empty(B, H, N, HEAD_DIM, **u8),
-                     torch.empty(B, H, N, HEAD_DIM, **u8), torch.empty(B, H, N // 64, **f32),
-                     torch.empty(B, H, N // 64, **f32), torch.empty(B, H, N // 64, **f32),
+                     torch.empty(B, H, N, HEAD_DIM, **u8), torch.empty(B, H, nb, **f32),
+                     torch.empty(B, H, nb, **f32), torch.empty(B, H, nb, **f32),
                      torch.empty(B, H, **f32), torch.empty(B, H, HEAD_DIM, **f32))
 
 

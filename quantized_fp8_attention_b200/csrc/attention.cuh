@@ -60,6 +60,10 @@ struct AttnParams {
   void* out;            // [B,H,N,128] BF16 or FP32
   int out_f32;
   uint32_t* status;     // device status word
+  const uint8_t* q8 = nullptr;       // FP8: the code tensors (read by the short-tile correction)
+  const uint8_t* k8 = nullptr;
+  const uint32_t* kmask = nullptr;   // FP8, key-masked kernel: excluded keys [B,H,ceil(N/32)]
+  float2* row_stats = nullptr;       // FP8, key-masked kernel: (m, l) per row [B,H,N]
 };
 
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {

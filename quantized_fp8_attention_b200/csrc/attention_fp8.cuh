@@ -37,6 +37,13 @@
 // of an item's last tile (each barrier counts one commit per issuer).  None
 // of these events waits on an MMA issued after it, so the fixed order cannot
 // deadlock; every wait is bounded.
+// Sequences of any length: the last KV tile of a head holds N % 128 keys.
+// The TMA loads (3-D: channel, row within the head, head) fill rows past N
+// with zeros; the K producer then overwrites the missing K rows of that tile
+// with copies of key N-1 (same scale block, so the same score: the row
+// maximum is unchanged), whose V rows stay zero (no term in O).  Their p
+// terms in the row sum are subtracted in the epilogue, from key N-1's score
+// recomputed from its codes.  The softmax loop itself carries no masking.
 #pragma once
 
 #include "attention.cuh"
@@ -61,8 +68,8 @@ struct F8Traits {
   static constexpr int kOffL = kOffP + 4 * kTileBytes;          // [item parity][tile][half][row]
   static constexpr int kOffBar = kOffL + 2 * 2 * 2 * 128 * 4;
   // fullK, fullV, emptyK, emptyV [kStages]; barQ, barQfree; barS, barSfree,
-  // barP, barPV, barDrain, barL [2 each]
-  static constexpr int kNumBars = 4 * kStages + 2 + 12;
+  // barP, barPV, barDrain, barL [2 each]; barPatch
+  static constexpr int kNumBars = 4 * kStages + 2 + 12 + 1;
   static constexpr int kSmemBytes = kOffBar + 8 * kNumBars + 16 + 1024;
 };
 
@@ -100,6 +107,39 @@ __device__ __forceinline__ float max32(const uint32_t (&u)[32]) {
   return fmax3(c0, __uint_as_float(u[15]), fmaxf(c1, __uint_as_float(u[31])));
 }
 
+// Absent keys of a KV tile (past the end of the sequence, or excluded by a key
+// mask): their scores in this thread's TMEM lane of S become -inf before the
+// softmax reads them, so they drop out of the row maximum and get p = 0 (with
+// a score scale a > 0, -inf * a = -inf).  pw<q>: bit k set when key 32q + k of
+// the tile is present.  Both threads of a row write the same values to the
+// same cells.
+__device__ __forceinline__ void mask_absent_scores(uint32_t tS, uint32_t pw0, uint32_t pw1, uint32_t pw2,
+                                                   uint32_t pw3) {
+#pragma unroll 1
+  for (int q = 0; q < 4; ++q) {
+    const uint32_t present = q == 0 ? pw0 : q == 1 ? pw1 : q == 2 ? pw2 : pw3;
+    if (present == ~0u) continue;
+    uint32_t v[32];
+    tmem_ld32(tS + 32u * (uint32_t)q, v);
+    tmem_wait_ld();
+#pragma unroll
+    for (int e = 0; e < 32; ++e)
+      if (!((present >> e) & 1u)) v[e] = 0xff800000u;
+    tmem_st32(tS + 32u * (uint32_t)q, v);
+  }
+  tmem_wait_st();
+}
+
+// kMaskable: some KV tiles may have absent keys -- the short last tile when N
+// is not a multiple of 128, and keys whose bit is set in p.kmask
+// ([B,H,ceil(N/32)] words, bit k of word w = key 32w + k; null = none) --
+// and each row's final maximum m and sum l go to p.row_stats (if not null).
+// Aligned calls without a mask use kMaskable = false, which holds no masking
+// code: the full-tile loop is the same instruction stream either way only
+// without it.
+// kShortTail: N is not a multiple of 128 (the patched short last tile above);
+// aligned calls use kShortTail = false and carry none of that code.
+template <bool kShortTail, bool kMaskable>
 __global__ void __launch_bounds__(kF8Threads, 1)
     attn_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
@@ -124,12 +164,14 @@ __global__ void __launch_bounds__(kF8Threads, 1)
   uint64_t* barPV = barQ + 8;      // [2] PV_t complete
   uint64_t* barDrain = barQ + 10;  // [2] error path: an issuer's MMAs completed
   uint64_t* barL = barQ + 12;      // [2] both halves' row sums written
+  uint64_t* barPatch = barQ + 14;  // the short last K tile landed (before its patch)
   float* sL = reinterpret_cast<float*>(smem + T::kOffL);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + T::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int N = p.N, nkv = N / kBlockN, nblk = N / 64;
+  const int N = p.N, nkv = (N + kBlockN - 1) / kBlockN, nblk = (N + 63) / 64;
+  const int valid_last = N - (nkv - 1) * kBlockN;   // keys in the last KV tile
   const int npairs = (N + 2 * kBlockM - 1) / (2 * kBlockM);
   const int nitems = p.B * p.H * npairs;
   // this CTA's items and KV tiles (tile g = local item * nkv + j)
@@ -146,6 +188,7 @@ __global__ void __launch_bounds__(kF8Threads, 1)
     }
     mbar_init(barQ, 1);
     mbar_init(barQfree, 2);
+    mbar_init(barPatch, 1);
     mbar_init(&barDrain[0], 1);
     mbar_init(&barDrain[1], 1);
     for (int t = 0; t < 2; ++t) {
@@ -181,22 +224,49 @@ __global__ void __launch_bounds__(kF8Threads, 1)
       if (is_k) tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(tm);
       int g = 0, pending = 0;
+      uint32_t patch_phase = 0;
       bool ok = true;
       for (int it = 0; ok && it < my_items; ++it) {
         const F8Item w = f8_item((int)blockIdx.x + it * (int)gridDim.x, p.H, npairs);
-        const int head_row = (w.b * p.H + w.h) * N;
+        const int head = w.b * p.H + w.h;
         if (is_k) {
           if (it > 0 && !(ok = mbar_wait(barQfree, (it - 1) & 1, abort_flag, p.status))) break;
           mbar_arrive_expect_tx(barQ, 2 * T::kTileBytes);
-          tma_load_2d(sQ, &tmQ, barQ, 0, head_row + w.qp * 2 * kBlockM);
-          tma_load_2d(sQ + T::kTileBytes, &tmQ, barQ, 0, head_row + w.qp * 2 * kBlockM + kBlockM);
+          tma_load_3d(sQ, &tmQ, barQ, 0, w.qp * 2 * kBlockM, head);
+          tma_load_3d(sQ + T::kTileBytes, &tmQ, barQ, 0, w.qp * 2 * kBlockM + kBlockM, head);
         }
         for (int j = 0; j < nkv; ++j, ++g) {
           const int s = g % T::kStages, r = g / T::kStages;
           if (!(ok = mbar_wait(&empty[s], (r & 1) ^ 1, abort_flag, p.status))) break;
-          mbar_arrive_expect_tx(&full[s], T::kTileBytes);
-          tma_load_2d(ring + s * T::kTileBytes, tm, &full[s], 0, head_row + j * kBlockN);
-          pending = g + 1;
+          uint8_t* dst = ring + s * T::kTileBytes;
+          if (kShortTail && is_k && j == nkv - 1) {
+            // the short last K tile: land it, then copy key N-1 (tile row
+            // valid_last - 1) over the zero-filled rows past N, and only then
+            // release it to the MMA.  Rows are 128 B with 16-byte chunk c of
+            // row x at c ^ (x % 8) (128-byte swizzle).
+            mbar_arrive_expect_tx(barPatch, T::kTileBytes);
+            tma_load_3d(dst, tm, barPatch, 0, j * kBlockN, head);
+            if (!(ok = mbar_wait(barPatch, patch_phase, abort_flag, p.status))) {
+              mbar_wait_drain(barPatch, patch_phase);
+              break;
+            }
+            patch_phase ^= 1u;
+            const int src = valid_last - 1;
+            uint4 row[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              row[c] = *reinterpret_cast<const uint4*>(dst + src * 128 + ((c ^ (src & 7)) << 4));
+            for (int x = valid_last; x < kBlockN; ++x)
+#pragma unroll
+              for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<uint4*>(dst + x * 128 + ((c ^ (x & 7)) << 4)) = row[c];
+            fence_proxy_async_smem();            // generic writes -> the MMA's reads
+            mbar_arrive(&full[s]);
+          } else {
+            mbar_arrive_expect_tx(&full[s], T::kTileBytes);
+            tma_load_3d(dst, tm, &full[s], 0, j * kBlockN, head);
+            pending = g + 1;
+          }
         }
       }
       if (*abort_flag) {
@@ -292,6 +362,7 @@ __global__ void __launch_bounds__(kF8Threads, 1)
     // row sits at c ^ (r % 8)
     const uint32_t prow = smem_u32(sP) + (uint32_t)(2 * t) * T::kTileBytes + (uint32_t)r * 128u;
     const uint32_t sw = (uint32_t)(r & 7);
+    const int nmw = (N + 31) / 32;               // key-mask words per head
     int g = 0;                                   // KV tile counter (global over items)
     bool ok = true;
     for (int it = 0; ok && it < my_items; ++it) {
@@ -302,20 +373,46 @@ __global__ void __launch_bounds__(kF8Threads, 1)
       const float* svp = p.sv + head * nblk;
       const float svmax = p.sv_max[head];
       const float a_row = p.sq[head * nblk + min(qrow, N - 1) / 64];
-      float sk0 = __ldg(skp), sk1 = __ldg(skp + 1), svh = __ldg(svp + hf);
+      // block scales of a tile; blocks past the end of a short sequence are
+      // read clamped (their keys are absent)
+      auto blk = [nblk](int J) { return (kShortTail && J >= nblk) ? nblk - 1 : J; };
+      float sk0 = __ldg(skp), sk1 = __ldg(skp + blk(1)), svh = __ldg(svp + blk(hf));
       float m = -INFINITY, l = 0.0f;
+
       for (int j = 0; j < nkv; ++j, ++g) {
         // block constants of this tile; the next tile's are loaded ahead
-        const float a0 = a_row * (sk0 * c_log2e), a1 = a_row * (sk1 * c_log2e);
-        const float ah = hf ? a1 : a0;
+        float a0 = a_row * (sk0 * c_log2e), a1 = a_row * (sk1 * c_log2e);
+        float ah = hf ? a1 : a0;
         const float cpv = svmax > 0.0f ? 448.0f * (svh / svmax) : 0.0f;
         if (j + 1 < nkv) {
           sk0 = __ldg(skp + 2 * j + 2);
-          sk1 = __ldg(skp + 2 * j + 3);
-          svh = __ldg(svp + 2 * j + 2 + hf);
+          sk1 = __ldg(skp + blk(2 * j + 3));
+          svh = __ldg(svp + blk(2 * j + 2 + hf));
         }
         if (!(ok = __all_sync(0xffffffffu, mbar_wait(&barS[t], g & 1, abort_flag, p.status)))) break;
         tc_fence_after();
+        if constexpr (kMaskable) {
+          // presence of the tile's keys, 32 per word: keys the caller's mask
+          // excludes (a short last tile is patched by the K producer)
+          uint32_t pw0 = ~0u, pw1 = ~0u, pw2 = ~0u, pw3 = ~0u;
+          if (p.kmask != nullptr) {
+            const uint32_t* km = p.kmask + head * nmw + 4 * j;
+            const int nw = nmw - 4 * j;
+            pw0 &= ~__ldg(km);
+            if (nw > 1) pw1 &= ~__ldg(km + 1);
+            if (nw > 2) pw2 &= ~__ldg(km + 2);
+            if (nw > 3) pw3 &= ~__ldg(km + 3);
+          }
+          if ((pw0 & pw1 & pw2 & pw3) != ~0u) {
+            mask_absent_scores(tS, pw0, pw1, pw2, pw3);
+            // -inf * 0 would be NaN: a zero scale becomes the smallest
+            // positive one, which gives the present keys the same p
+            // (x = S * 2^-149 is absorbed by x - m, or is 0 when S is)
+            a0 = fmaxf(a0, 1.401298464e-45f);
+            a1 = fmaxf(a1, 1.401298464e-45f);
+            ah = hf ? a1 : a0;
+          }
+        }
         // raw maxima of the other half (its scores are not kept) and of this
         // half; the first 32 of this half's scores stay in registers, the
         // other 32 are read again when the exponential loop gets to them.
@@ -341,7 +438,9 @@ __global__ void __launch_bounds__(kF8Threads, 1)
         // zero) is the rounded product of the raw max
         const float h0 = hf ? mo : mh, h1 = hf ? mh : mo;
         const float m_new = fmaxf(m, fmaxf(__fmul_rz(h0, a0), __fmul_rz(h1, a1)));
-        const float alpha = ex2_approx(m - m_new);
+        // a tile with no key present, after tiles with none, leaves
+        // m = m_new = -inf with nothing to rescale (key masks only)
+        const float alpha = (kMaskable && m_new == -INFINITY) ? 1.0f : ex2_approx(m - m_new);
         const float2 nm2 = make_float2(-m_new, -m_new);
         const float2 a2 = make_float2(ah, ah);
         float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
@@ -415,12 +514,37 @@ __global__ void __launch_bounds__(kF8Threads, 1)
       lx[hf * 128 + r] = l;
       mbar_arrive(&barL[t]);
       if (!(ok = __all_sync(0xffffffffu, mbar_wait(&barL[t], it & 1, abort_flag, p.status)))) break;
-      const float l_row = lx[r] + lx[128 + r];
+      float l_row = lx[r] + lx[128 + r];
+      if (kShortTail && qrow < N) {
+        // the copies of key N-1 in the short last tile added 128 - valid_last
+        // terms p(N-1) = 2^(x - m) to l: recompute key N-1's score from the
+        // codes (E4M3 products are exact in binary32) and take them out
+        const uint32_t* qa = reinterpret_cast<const uint32_t*>(p.q8 + (head * N + qrow) * 128);
+        const uint32_t* ka = reinterpret_cast<const uint32_t*>(p.k8 + (head * N + N - 1) * 128);
+        float sdot = 0.0f;
+#pragma unroll 4
+        for (int c4 = 0; c4 < 32; ++c4) {
+          const uint32_t qw = __ldg(qa + c4), kw = __ldg(ka + c4);
+          const float2 q01 = e4m3x2_to_f2(qw & 0xFFFFu), q23 = e4m3x2_to_f2(qw >> 16);
+          const float2 k01 = e4m3x2_to_f2(kw & 0xFFFFu), k23 = e4m3x2_to_f2(kw >> 16);
+          sdot = __fmaf_rn(q01.x, k01.x, sdot);
+          sdot = __fmaf_rn(q01.y, k01.y, sdot);
+          sdot = __fmaf_rn(q23.x, k23.x, sdot);
+          sdot = __fmaf_rn(q23.y, k23.y, sdot);
+        }
+        const float a_last = a_row * (__ldg(skp + nblk - 1) * c_log2e);
+        const float p_dup = ex2_approx(__fmaf_rn(__fmul_rz(sdot, a_last), 1.0f, -m));
+        l_row -= (float)(kBlockN - valid_last) * p_dup;
+      }
       if (!(ok = __all_sync(0xffffffffu, mbar_wait(&barPV[t], (g - 1) & 1, abort_flag, p.status)))) break;
       tc_fence_after();
       const bool store = qrow < N;
-      const float fin = (svmax / 448.0f) / l_row;
+      // l_row = 0 only when a key mask excluded every key of the row
+      const float fin = (kMaskable && !(l_row > 0.0f)) ? 0.0f : (svmax / 448.0f) / l_row;
       const size_t orow = head * N + (size_t)qrow;
+      if constexpr (kMaskable) {
+        if (p.row_stats != nullptr && hf == 0 && store) p.row_stats[orow] = make_float2(m, l_row);
+      }
 #pragma unroll 1
       for (int c = 0; c < 2; ++c) {
         uint32_t o[32];

@@ -22,6 +22,9 @@
 // commit that signals S_t(j+1) also covers PV_t(j), so once softmax t sees
 // S_t(j+1) it may rescale O_t.  The two softmax warpgroups take turns for
 // their exponential loops.
+// Sequences of any length: TMA loads are 3-D (channel, row within the head,
+// head), rows past N read as zeros, and the last KV tile's keys past N get
+// raw score -inf, so p = 0 for them (the scale here is always > 0).
 #pragma once
 
 #include "attention.cuh"
@@ -105,7 +108,8 @@ __global__ void __launch_bounds__(kWsThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int N = p.N, nkv = N / kBlockN;
+  const int N = p.N, nkv = (N + kBlockN - 1) / kBlockN;
+  const int valid_last = N - (nkv - 1) * kBlockN;   // keys in the last KV tile
   const int npairs = (N + kPairRows - 1) / kPairRows;
   const int nitems = p.B * p.H * npairs;
   const float c_log2e = p.softmax_scale * 1.4426950408889634f;
@@ -146,28 +150,28 @@ __global__ void __launch_bounds__(kWsThreads, 1)
       bool ok = true;
       for (int item = blockIdx.x; ok && item < nitems; item += gridDim.x, ++it) {
         const WsItem w = ws_item(item, p.H, npairs);
-        const int head_row = (w.b * p.H + w.h) * N;
+        const int head = w.b * p.H + w.h;
         if (it > 0 && !(ok = mbar_wait(barQfree, (it - 1) & 1, abort_flag, p.status))) break;
         mbar_arrive_expect_tx(barQ, 2 * T::kTileBytes);
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
-          const int y = head_row + w.qp * kPairRows + t * kBlockM;
+          const int y = w.qp * kPairRows + t * kBlockM;
           uint8_t* dst = sQ + t * T::kTileBytes;
-          tma_load_2d(dst, &tmQ, barQ, 0, y);
-          tma_load_2d(dst + 16384, &tmQ, barQ, 64, y);
+          tma_load_3d(dst, &tmQ, barQ, 0, y, head);
+          tma_load_3d(dst + 16384, &tmQ, barQ, 64, y, head);
         }
         for (int j = 0; j < nkv; ++j, ++g) {
           const int s = g % T::kStages, r = g / T::kStages;
           if (!(ok = mbar_wait(&empty[s], (r & 1) ^ 1, abort_flag, p.status))) break;
-          const int y = head_row + j * kBlockN;
+          const int y = j * kBlockN;
           mbar_arrive_expect_tx(&fullK[s], T::kTileBytes);
           mbar_arrive_expect_tx(&fullV[s], T::kTileBytes);
           uint8_t* dk = sK + s * T::kTileBytes;
           uint8_t* dv = sV + s * T::kTileBytes;
-          tma_load_2d(dk, &tmK, &fullK[s], 0, y);
-          tma_load_2d(dv, &tmV, &fullV[s], 0, y);
-          tma_load_2d(dk + 16384, &tmK, &fullK[s], 64, y);
-          tma_load_2d(dv + 16384, &tmV, &fullV[s], 64, y);
+          tma_load_3d(dk, &tmK, &fullK[s], 0, y, head);
+          tma_load_3d(dv, &tmV, &fullV[s], 0, y, head);
+          tma_load_3d(dk + 16384, &tmK, &fullK[s], 64, y, head);
+          tma_load_3d(dv + 16384, &tmV, &fullV[s], 64, y, head);
           pending = g + 1;
         }
       }
@@ -275,6 +279,14 @@ __global__ void __launch_bounds__(kWsThreads, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld32(tS + lane_off + 32u * c, sr[c]);
         tmem_wait_ld();
+        if (j == nkv - 1 && valid_last < kBlockN) {
+          // keys past the end of the sequence: raw score -inf, so p = 0
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (32 * c + e >= valid_last) sr[c][e] = 0xff800000u;
+        }
         const float a0 = c_log2e, a1 = c_log2e;
         // maxima of the raw scores per 64-key half (8 independent chains);
         // the scales are >= 0 and rounding is monotone, so the tile max of

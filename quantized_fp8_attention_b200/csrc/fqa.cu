@@ -73,17 +73,19 @@ static EncodeTiledFn encoder() {
   return g_encode;
 }
 
-// 2-D view [rows, 128] of a [B,H,N,128] tensor; box = 128 rows x (128 B of
-// columns), 128-byte swizzle.
-static bool make_tmap(CUtensorMap* m, const void* base, bool fp8, uint64_t rows) {
+// 3-D view (channel, row within the head, head) of a [B,H,N,128] tensor; box
+// = 128 B of channels x 128 rows x 1 head, 128-byte swizzle.  Rows past N
+// (the short last tile of a sequence) are filled with zeros, never read from
+// the next head.
+static bool make_tmap(CUtensorMap* m, const void* base, bool fp8, int N, int heads) {
   EncodeTiledFn enc = encoder();
   if (!enc) return false;
   const uint32_t elt = fp8 ? 1 : 2;
-  cuuint64_t dims[2] = {128, rows};
-  cuuint64_t strides[1] = {128ull * elt};
-  cuuint32_t box[2] = {128u / elt, 128u};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+  cuuint64_t dims[3] = {128, (cuuint64_t)N, (cuuint64_t)heads};
+  cuuint64_t strides[2] = {128ull * elt, 128ull * elt * (cuuint64_t)N};
+  cuuint32_t box[3] = {128u / elt, 128u, 1u};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
                    const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -92,11 +94,12 @@ static bool make_tmap(CUtensorMap* m, const void* base, bool fp8, uint64_t rows)
 
 static bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-// Shape checks shared by every call. n_mult: required multiple of N.
-static fqa_status check_shape(int B, int H, int N, int d, int n_mult) {
+// Shape checks shared by every call: any N >= 1 (the last 64-token block and
+// the last 128-key tile of a head may be short).
+static fqa_status check_shape(int B, int H, int N, int d) {
   if (B < 1 || H < 1 || N < 1 || d < 1) return FQA_ERR_INVALID_ARG;
   if (d != 128) return FQA_ERR_UNSUPPORTED;
-  if (N % n_mult != 0 || N > 65536) return FQA_ERR_UNSUPPORTED;
+  if (N > 65536) return FQA_ERR_UNSUPPORTED;
   if ((int64_t)B * H > 65535) return FQA_ERR_UNSUPPORTED;
   if ((int64_t)B * H * N >= (int64_t(1) << 31)) return FQA_ERR_UNSUPPORTED;
   return FQA_OK;
@@ -117,10 +120,10 @@ static int num_sms() {
 // BF16: persistent launch, one CTA per SM (or per work item, if fewer).
 static fqa_status launch_attention_bf16(const void* q, const void* k, const void* v,
                                         const AttnParams& prm, cudaStream_t stream) {
-  const uint64_t rows = (uint64_t)prm.B * prm.H * prm.N;
+  const int heads = prm.B * prm.H;
   CUtensorMap tq, tk, tv;
-  if (!make_tmap(&tq, q, false, rows) || !make_tmap(&tk, k, false, rows) ||
-      !make_tmap(&tv, v, false, rows))
+  if (!make_tmap(&tq, q, false, prm.N, heads) || !make_tmap(&tk, k, false, prm.N, heads) ||
+      !make_tmap(&tv, v, false, prm.N, heads))
     return FQA_ERR_CUDA;
   if (cudaFuncSetAttribute(attn_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            BfTraits::kSmemBytes) != cudaSuccess)
@@ -137,19 +140,27 @@ static fqa_status launch_attention_bf16(const void* q, const void* k, const void
 // per work item, if fewer).
 static fqa_status launch_attention_fp8(const void* q, const void* k, const void* v,
                                        const AttnParams& prm, cudaStream_t stream) {
-  const uint64_t rows = (uint64_t)prm.B * prm.H * prm.N;
+  const int heads = prm.B * prm.H;
   CUtensorMap tq, tk, tv;
-  if (!make_tmap(&tq, q, true, rows) || !make_tmap(&tk, k, true, rows) ||
-      !make_tmap(&tv, v, true, rows))
+  if (!make_tmap(&tq, q, true, prm.N, heads) || !make_tmap(&tk, k, true, prm.N, heads) ||
+      !make_tmap(&tv, v, true, prm.N, heads))
     return FQA_ERR_CUDA;
-  if (cudaFuncSetAttribute(attn_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  // the instance that carries only what the call needs: the short-tail patch
+  // when N is not a multiple of 128, the key mask and row statistics when
+  // given
+  const bool tail = prm.N % kBlockN != 0;
+  const bool masked = prm.kmask != nullptr || prm.row_stats != nullptr;
+  using KernelFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const AttnParams);
+  const KernelFn fn = tail ? (masked ? attn_fp8_kernel<true, true> : attn_fp8_kernel<true, false>)
+                           : (masked ? attn_fp8_kernel<false, true> : attn_fp8_kernel<false, false>);
+  if (cudaFuncSetAttribute((const void*)fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            F8Traits::kSmemBytes) != cudaSuccess)
     return FQA_ERR_CUDA;
   const int items = prm.B * prm.H * ((prm.N + 2 * kBlockM - 1) / (2 * kBlockM));
   const int sms = num_sms();
   if (sms <= 0) return FQA_ERR_CUDA;
   const int grid = items < sms ? items : sms;
-  attn_fp8_kernel<<<grid, kF8Threads, F8Traits::kSmemBytes, stream>>>(tq, tk, tv, prm);
+  fn<<<grid, kF8Threads, F8Traits::kSmemBytes, stream>>>(tq, tk, tv, prm);
   return launch_status();
 }
 
@@ -173,14 +184,15 @@ const char* fqa_status_string(fqa_status s) {
   return "FQA_UNKNOWN_STATUS";
 }
 
-// Workspace: the K-mean partial sums [B,H,N/64,128] FP32, then (256-byte
-// aligned) the grid-barrier counter of the fused quantize launch.
+// Workspace: the K-mean partial sums [B,H,ceil(N/64),128] FP32, then
+// (256-byte aligned) the grid-barrier and work-queue counters of the fused
+// quantize launch.
 static size_t partial_bytes(int B, int H, int N, int d) {
-  return (size_t)B * H * (N / kQBlock) * d * sizeof(float);
+  return (size_t)B * H * ((N + kQBlock - 1) / kQBlock) * d * sizeof(float);
 }
 
 size_t fqa_quantize_workspace_bytes(int B, int H, int N, int d) {
-  if (check_shape(B, H, N, d, kQBlock) != FQA_OK) return 0;
+  if (check_shape(B, H, N, d) != FQA_OK) return 0;
   return ((partial_bytes(B, H, N, d) + 255) & ~size_t(255)) + 256;
 }
 
@@ -188,7 +200,7 @@ fqa_status fqa_quantize(const void* q, const void* k, const void* v, int B, int 
                         void* q8, void* k8, void* v8, float* sq, float* sk, float* sv,
                         float* sv_max, float* k_mean, void* workspace, size_t workspace_bytes,
                         void* cuda_stream) {
-  fqa_status st = check_shape(B, H, N, d, kQBlock);
+  fqa_status st = check_shape(B, H, N, d);
   if (st != FQA_OK) return st;
   const void* ptrs[] = {q, k, v, q8, k8, v8, sq, sk, sv, sv_max, k_mean, workspace};
   for (const void* p : ptrs)
@@ -206,7 +218,7 @@ fqa_status fqa_quantize(const void* q, const void* k, const void* v, int B, int 
   float* partial = static_cast<float*>(workspace);
   unsigned int* ctr = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(workspace) +
                                                       ((partial_bytes(B, H, N, d) + 255) & ~size_t(255)));
-  const int nunits = B * H * (N / kQBlock);
+  const int nunits = B * H * ((N + kQBlock - 1) / kQBlock);
   if (cudaFuncSetAttribute(quantize_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            kQuantSmem) != cudaSuccess)
     return FQA_ERR_CUDA;
@@ -238,7 +250,7 @@ fqa_status fqa_quantize(const void* q, const void* k, const void* v, int B, int 
 
 static fqa_status check_attention_common(int B, int H, int N, int d, float softmax_scale,
                                          void* out, fqa_out_dtype out_dtype) {
-  fqa_status st = check_shape(B, H, N, d, kBlockN);
+  fqa_status st = check_shape(B, H, N, d);
   if (st != FQA_OK) return st;
   if (!(std::isfinite(softmax_scale) && softmax_scale > 0.0f)) return FQA_ERR_INVALID_ARG;
   if (out == nullptr) return FQA_ERR_INVALID_ARG;
@@ -265,6 +277,10 @@ fqa_status fqa_attention_fp8(const void* q8, const void* k8, const void* v8, con
   uint32_t* status = status_ptr(&st);
   if (!status) return st;
   AttnParams prm{B, H, N, softmax_scale, sq, sk, sv, sv_max, out, out_dtype == FQA_OUT_F32, status};
+  prm.q8 = static_cast<const uint8_t*>(q8);
+  prm.k8 = static_cast<const uint8_t*>(k8);
+  prm.kmask = nullptr;
+  prm.row_stats = nullptr;
   return launch_attention_fp8(q8, k8, v8, prm, static_cast<cudaStream_t>(cuda_stream));
 }
 
@@ -368,7 +384,7 @@ extern "C" fqa_status fqa_quantize_noalloc(const void* q, const void* k, const v
                                            int N, int d, void* q8, void* k8, void* v8, float* sq,
                                            float* sk, float* sv, float* sv_max, float* k_mean,
                                            void* cuda_stream) {
-  fqa_status st = check_shape(B, H, N, d, kQBlock);
+  fqa_status st = check_shape(B, H, N, d);
   if (st != FQA_OK) return st;
   if (fqa_quantize_workspace_bytes(B, H, N, d) > kNoAllocScratchBytes) return FQA_ERR_UNSUPPORTED;
   float* scratch = noalloc_scratch(&st);

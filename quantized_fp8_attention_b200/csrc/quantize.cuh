@@ -10,10 +10,13 @@
 //             (sum over the block's tokens ascending of k[n][c])) / N,
 //            every sum a sequential binary32 sum from +0, one RN division;
 //   x      = q, fl32(k - mu[c]) or v;
-//   amax   = max |x| over the block's 64 x 128 values;
+//   amax   = max |x| over the block's (at most 64) x 128 values;
 //   s      = amax / 448, inv = 448 / amax (RN divisions; 0 and 0 if amax = 0);
-//   code   = E4M3_RNE_satfinite(fl32(x * inv));
+//   code   = E4M3_RNE_satfinite(fl32(x * inv))   (x / s where inv overflows,
+//            signed zeros where s underflows);
 //   sv_max = max over the head's V block scales.
+// Any N >= 1: the last block of a head holds the N - 64*(ceil(N/64)-1)
+// remaining tokens, and its scale is their absmax alone.
 // Inputs are BF16 [B,H,N,128]; codes are written in the same layout.
 #pragma once
 
@@ -31,8 +34,8 @@ namespace fqa {
 //       the V unit scales (no atomics)
 //   3   K units -> smoothed codes and scales, newest units of 1b first (each
 //       unit's head mean row arrives with the unit)
-// Unit u = (b*H + h)*(N/64) + j is one 64-token block of one head: 16 KB of
-// contiguous BF16 per tensor.  Units are handed out through work queues
+// Unit u = (b*H + h)*ceil(N/64) + j is one 64-token block of one head: 16 KB
+// of contiguous BF16 per tensor (the last block of a head may be shorter).  Units are handed out through work queues
 // (counters the launch zeroes), so the SMs that stream faster take more.
 // All loads are 1-D bulk copies into a shared-memory ring of kRingBytes, cut
 // into as many slots as the phase's unit size allows, so each SM keeps several
@@ -89,11 +92,13 @@ __device__ __forceinline__ bool grid_barrier(unsigned int* ctr, unsigned int rou
   return *failed == 0;
 }
 
-// The values of this thread's chunks of a staged BF16 unit.
-__device__ __forceinline__ void chunks_to_f32(const uint8_t* blk, float (&x)[kVals]) {
+// The values of this thread's chunks of a staged BF16 unit; chunks at or
+// beyond nvalid (past a short block's tokens) read as zeros.
+__device__ __forceinline__ void chunks_to_f32(const uint8_t* blk, int nvalid, float (&x)[kVals]) {
 #pragma unroll
   for (int i = 0; i < kChunks; ++i) {
-    const uint4 raw = *reinterpret_cast<const uint4*>(blk + 16 * (threadIdx.x + kQuantThreads * i));
+    const int c = threadIdx.x + kQuantThreads * i;
+    const uint4 raw = c < nvalid ? *reinterpret_cast<const uint4*>(blk + 16 * c) : make_uint4(0, 0, 0, 0);
     const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
@@ -105,9 +110,10 @@ __device__ __forceinline__ void chunks_to_f32(const uint8_t* blk, float (&x)[kVa
 }
 
 // Block absmax over the CTA (red: one float per warp for this slot), scale,
-// and the codes of this thread's chunks (8 bytes per chunk, chunk c at byte 8c).
+// and the codes of this thread's chunks (8 bytes per chunk, chunk c at byte
+// 8c; chunks at or beyond nvalid are not stored).
 __device__ __forceinline__ float quantize_chunks(float (&x)[kVals], float* red, uint8_t* dst, int slot,
-                                                 uint64_t policy) {
+                                                 int nvalid, uint64_t policy) {
   const int t = threadIdx.x;
   float m = 0.0f;
 #pragma unroll
@@ -131,7 +137,8 @@ __device__ __forceinline__ float quantize_chunks(float (&x)[kVals], float* red, 
 #pragma unroll
       for (int e = 0; e < 4; ++e)
         w[e] = e4m3x2(__fdiv_rn(x[8 * i + 2 * e], scale), __fdiv_rn(x[8 * i + 2 * e + 1], scale));
-      st_global_v2_hint(dst + 8 * (t + kQuantThreads * i), w[0] | (w[1] << 16), w[2] | (w[3] << 16), policy);
+      if (t + kQuantThreads * i < nvalid)
+        st_global_v2_hint(dst + 8 * (t + kQuantThreads * i), w[0] | (w[1] << 16), w[2] | (w[3] << 16), policy);
     }
     return scale;
   }
@@ -141,7 +148,8 @@ __device__ __forceinline__ float quantize_chunks(float (&x)[kVals], float* red, 
     uint32_t hi = e4m3x2(__fmul_rn(x[8 * i + 2], inv), __fmul_rn(x[8 * i + 3], inv));
     uint32_t lo2 = e4m3x2(__fmul_rn(x[8 * i + 4], inv), __fmul_rn(x[8 * i + 5], inv));
     uint32_t hi2 = e4m3x2(__fmul_rn(x[8 * i + 6], inv), __fmul_rn(x[8 * i + 7], inv));
-    st_global_v2_hint(dst + 8 * (t + kQuantThreads * i), lo | (hi << 16), lo2 | (hi2 << 16), policy);
+    if (t + kQuantThreads * i < nvalid)
+      st_global_v2_hint(dst + 8 * (t + kQuantThreads * i), lo | (hi << 16), lo2 | (hi2 << 16), policy);
   }
   return scale;
 }
@@ -160,7 +168,7 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantMinCtas) quantize_fused_k
   __shared__ float red[2 * kQuantWarps];
   __shared__ int failed, abort_flag;
   const int t = threadIdx.x;
-  const int nblk = N / kQBlock;
+  const int nblk = (N + kQBlock - 1) / kQBlock;
   const int nunits = B * H * nblk;
   const int G = gridDim.x;
   if (t == 0) {
@@ -220,24 +228,29 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantMinCtas) quantize_fused_k
       return reverse ? nunits - 1 - (int)i : (int)i;
     };
   };
-  auto blk_ptr = [&](const __nv_bfloat16* base, int u) {
-    return base + (size_t)u * kQBlock * kHeadDim;
+  // element offset of unit u in a [B,H,N,128] tensor, and its token count
+  auto unit_off = [&](int u) {
+    const int hd = u / nblk;
+    return ((size_t)hd * N + (size_t)(u - hd * nblk) * kQBlock) * kHeadDim;
   };
+  auto unit_rows = [&](int u) { return min(kQBlock, N - (u % nblk) * kQBlock); };
 
   // ---- phase 1a: Q and V (streamed once: evict-first)
   bool ok = run(2 * kBlockBytes, queue(kCtrQV, false),
       [&](int u, uint8_t* dst, uint64_t* bar) {
-        mbar_arrive_expect_tx(bar, 2 * kBlockBytes);
-        bulk_load(dst, blk_ptr(q, u), kBlockBytes, bar, pol_first);
-        bulk_load(dst + kBlockBytes, blk_ptr(v, u), kBlockBytes, bar, pol_first);
+        const uint32_t bytes = (uint32_t)unit_rows(u) * kHeadDim * 2;
+        mbar_arrive_expect_tx(bar, 2 * bytes);
+        bulk_load(dst, q + unit_off(u), bytes, bar, pol_first);
+        bulk_load(dst + kBlockBytes, v + unit_off(u), bytes, bar, pol_first);
       },
       [&](int u, const uint8_t* blk) {
-        const size_t off = (size_t)u * kQBlock * kHeadDim;
+        const size_t off = unit_off(u);
+        const int nvalid = unit_rows(u) * (kHeadDim * 2 / 16);
         float x[kVals];
-        chunks_to_f32(blk, x);
-        const float s_q = quantize_chunks(x, red, q8 + off, 0, pol_first);
-        chunks_to_f32(blk + kBlockBytes, x);
-        const float s_v = quantize_chunks(x, red, v8 + off, 1, pol_first);
+        chunks_to_f32(blk, nvalid, x);
+        const float s_q = quantize_chunks(x, red, q8 + off, 0, nvalid, pol_first);
+        chunks_to_f32(blk + kBlockBytes, nvalid, x);
+        const float s_v = quantize_chunks(x, red, v8 + off, 1, nvalid, pol_first);
         if (t == 0) {
           sq[u] = s_q;
           sv[u] = s_v;
@@ -248,15 +261,21 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantMinCtas) quantize_fused_k
   if (ok)
     ok = run(kBlockBytes, queue(kCtrK, false),
         [&](int u, uint8_t* dst, uint64_t* bar) {
-          mbar_arrive_expect_tx(bar, kBlockBytes);
-          bulk_load(dst, blk_ptr(k, u), kBlockBytes, bar, pol_last);
+          const uint32_t bytes = (uint32_t)unit_rows(u) * kHeadDim * 2;
+          mbar_arrive_expect_tx(bar, bytes);
+          bulk_load(dst, k + unit_off(u), bytes, bar, pol_last);
         },
         [&](int u, const uint8_t* blk) {
           if (t < kHeadDim) {
             const __nv_bfloat16* kb = reinterpret_cast<const __nv_bfloat16*>(blk);
+            const int rows = unit_rows(u);
             float acc = 0.0f;
+            if (rows == kQBlock) {
 #pragma unroll 16
-            for (int n = 0; n < kQBlock; ++n) acc = __fadd_rn(acc, __bfloat162float(kb[n * kHeadDim + t]));
+              for (int n = 0; n < kQBlock; ++n) acc = __fadd_rn(acc, __bfloat162float(kb[n * kHeadDim + t]));
+            } else {
+              for (int n = 0; n < rows; ++n) acc = __fadd_rn(acc, __bfloat162float(kb[n * kHeadDim + t]));
+            }
             partial[(size_t)u * kHeadDim + t] = acc;
           }
         });
@@ -314,8 +333,9 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantMinCtas) quantize_fused_k
   constexpr int kSlot3 = kBlockBytes + kHeadDim * 4;
   run(kSlot3, queue(kCtrK3, true),
       [&](int u, uint8_t* dst, uint64_t* bar) {
-        mbar_arrive_expect_tx(bar, kSlot3);
-        bulk_load(dst, blk_ptr(k, u), kBlockBytes, bar, pol_first);
+        const uint32_t bytes = (uint32_t)unit_rows(u) * kHeadDim * 2;
+        mbar_arrive_expect_tx(bar, bytes + kHeadDim * 4);
+        bulk_load(dst, k + unit_off(u), bytes, bar, pol_first);
         bulk_load(dst + kBlockBytes, k_mean + (size_t)(u / nblk) * kHeadDim, kHeadDim * 4, bar, pol_first);
       },
       [&](int u, const uint8_t* blk) {
@@ -324,13 +344,18 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantMinCtas) quantize_fused_k
         float mr[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) mr[e] = mu[e];
+        const int nvalid = unit_rows(u) * (kHeadDim * 2 / 16);
         float x[kVals];
-        chunks_to_f32(blk, x);
+        chunks_to_f32(blk, nvalid, x);
 #pragma unroll
-        for (int i4 = 0; i4 < kChunks; ++i4)
+        for (int i4 = 0; i4 < kChunks; ++i4) {
+          // chunks past a short block's tokens stay 0: they must not enter amax
+          if (t + kQuantThreads * i4 < nvalid) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) x[8 * i4 + e] = __fsub_rn(x[8 * i4 + e], mr[e]);
-        const float s_k = quantize_chunks(x, red, k8 + (size_t)u * kQBlock * kHeadDim, 0, pol_first);
+            for (int e = 0; e < 8; ++e) x[8 * i4 + e] = __fsub_rn(x[8 * i4 + e], mr[e]);
+          }
+        }
+        const float s_k = quantize_chunks(x, red, k8 + unit_off(u), 0, nvalid, pol_first);
         if (t == 0) sk[u] = s_k;
       });
 }

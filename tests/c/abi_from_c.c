@@ -21,7 +21,8 @@ int main(void) {
   CHECK(fqa_status_string(FQA_ERR_TIMEOUT) != fqa_status_string(FQA_OK));
   /* B*H*(N/64)*d*4 rounded up to 256, plus 256 bytes of counters */
   CHECK(fqa_quantize_workspace_bytes(1, 24, 8704, 128) == 1671168 + 256);
-  CHECK(fqa_quantize_workspace_bytes(1, 1, 100, 128) == 0);
+  CHECK(fqa_quantize_workspace_bytes(1, 1, 100, 128) == 1024 + 256); /* a short last block */
+  CHECK(fqa_quantize_workspace_bytes(1, 1, 100, 64) == 0);
   /* 8 MiB of partial sums plus the 256 counter bytes: exactly 16384 blocks fit */
   CHECK(fqa_quantize_noalloc_max_workspace_bytes() == ((size_t)8 << 20) + 256);
   CHECK(fqa_quantize_workspace_bytes(1, 16, 65536, 128) == fqa_quantize_noalloc_max_workspace_bytes());
@@ -32,7 +33,7 @@ int main(void) {
         FQA_ERR_INVALID_ARG);
   CHECK(fqa_quantize(p, p, p, 1, 1, 128, 64, p, p, p, f, f, f, f, f, p, 1 << 20, NULL) ==
         FQA_ERR_UNSUPPORTED);
-  CHECK(fqa_attention_fp8(p, p, p, f, f, f, f, 1, 1, 192, 128, 0.088f, p, FQA_OUT_BF16, NULL) ==
+  CHECK(fqa_attention_fp8(p, p, p, f, f, f, f, 1, 1, 192, 64, 0.088f, p, FQA_OUT_BF16, NULL) ==
         FQA_ERR_UNSUPPORTED);
   CHECK(fqa_attention_bf16(p, p, p, 1, 1, 128, 128, -1.0f, p, FQA_OUT_BF16, NULL) ==
         FQA_ERR_INVALID_ARG);

@@ -47,11 +47,14 @@ def test_status_strings_and_version(L):
 def test_workspace_bytes(L):
     import quantized_fp8_attention_b200 as fqa
     r256 = lambda x: (x + 255) // 256 * 256
-    ws = lambda B, H, N: r256(B * H * (N // 64) * 128 * 4) + 256
+    ws = lambda B, H, N: r256(B * H * ((N + 63) // 64) * 128 * 4) + 256
     assert fqa.fqa_quantize_workspace_bytes(1, 24, 8704) == ws(1, 24, 8704) == 1671168 + 256
     assert fqa.fqa_quantize_workspace_bytes(2, 24, 16896) == ws(2, 24, 16896)
     assert fqa.fqa_quantize_workspace_bytes(1, 65535, 64) == ws(1, 65535, 64)
-    assert fqa.fqa_quantize_workspace_bytes(1, 1, 100) == 0       # N % 64 != 0
+    assert fqa.fqa_quantize_workspace_bytes(1, 1, 100) == ws(1, 1, 100) == 1024 + 256   # short last block
+    assert fqa.fqa_quantize_workspace_bytes(1, 1, 1) == 512 + 256
+    assert fqa.fqa_quantize_workspace_bytes(1, 1, 0) == 0
+    assert fqa.fqa_quantize_workspace_bytes(1, 1, 65537) == 0     # N > 65536
     assert fqa.fqa_quantize_workspace_bytes(1, 1, 128, 64) == 0   # d != 128
 
 
@@ -72,7 +75,7 @@ def test_quantize_validation(L):
     assert L.fqa_quantize(*args(ws=None)) == 1
     assert L.fqa_quantize(*args(B=0)) == 1
     assert L.fqa_quantize(*args(d=64)) == 2
-    assert L.fqa_quantize(*args(N=96)) == 2
+    assert L.fqa_quantize(*args(N=0)) == 1
     assert L.fqa_quantize(*args(N=65600)) == 2
     assert L.fqa_quantize(*args(B=300, H=300)) == 2
     assert L.fqa_quantize(*args(wsb=16)) == 1
@@ -95,14 +98,15 @@ def test_attention_validation(L):
     assert fp8(scale=0.0) == 1
     assert fp8(scale=float("inf")) == 1
     assert fp8(dt=5) == 1
-    assert fp8(N=64) == 2
+    assert fp8(N=65537) == 2
+    assert fp8(N=0) == 1
     assert fp8(d=256) == 2
     assert fp8(v8=_p(0x10001)) == 3
     assert fp8(out=_p(0x10004)) == 3
     bf = lambda **kw: L.fqa_attention_bf16(kw.get("q", ok), ok, ok, 1, 1, kw.get("N", 128), 128,
                                            f(kw.get("scale", 0.088)), kw.get("out", ok), 0, None)
     assert bf(q=None) == 1
-    assert bf(N=200) == 2
+    assert bf(N=70000) == 2
     assert bf(scale=-1.0) == 1
     assert bf(q=_p(0x10002)) == 3
     assert L.fqa_e4m3_encode(None, ok, 4, None) == 1

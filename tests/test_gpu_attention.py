@@ -207,7 +207,7 @@ def test_fp8_deterministic():
 
 def test_attention_rejects_bad_arguments():
     fqa = _fqa()
-    t = torch.zeros(1, 1, 192, 128, dtype=torch.uint8, device="cuda")   # N % 128 != 0
+    t = torch.zeros(1, 1, 192, 64, dtype=torch.uint8, device="cuda")    # d != 128
     s = torch.ones(1, 1, 3, device="cuda")
     sm = torch.ones(1, 1, device="cuda")
     out = torch.empty(1, 1, 192, 128, dtype=torch.bfloat16, device="cuda")

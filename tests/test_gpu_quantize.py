@@ -53,8 +53,8 @@ def test_quantize_deterministic_and_canaries():
         holders = []
         parts = []
         for shape, dt, fill in (((B, H, N, 128), torch.uint8, 0xA5), ((B, H, N, 128), torch.uint8, 0xA5),
-                                ((B, H, N, 128), torch.uint8, 0xA5), ((B, H, N // 64), torch.float32, -7.0),
-                                ((B, H, N // 64), torch.float32, -7.0), ((B, H, N // 64), torch.float32, -7.0),
+                                ((B, H, N, 128), torch.uint8, 0xA5), ((B, H, fqa.nblocks(N)), torch.float32, -7.0),
+                                ((B, H, fqa.nblocks(N)), torch.float32, -7.0), ((B, H, fqa.nblocks(N)), torch.float32, -7.0),
                                 ((B, H), torch.float32, -7.0), ((B, H, 128), torch.float32, -7.0)):
             base, view = guarded(shape, dt, fill)
             holders.append((base, view.numel(), fill))
@@ -94,7 +94,7 @@ def test_quantize_edge_blocks():
 
 def test_quantize_rejects_bad_arguments():
     fqa = _fqa()
-    t = torch.zeros(1, 1, 100, 128, dtype=torch.bfloat16, device="cuda")   # N % 64 != 0
+    t = torch.zeros(1, 1, 100, 64, dtype=torch.bfloat16, device="cuda")    # d != 128
     qz = fqa.alloc_quantized(1, 1, 128, "cuda")
     ws = fqa.alloc_workspace(1, 1, 128, "cuda")
     assert fqa.fqa_quantize(t, t, t, *qz, ws) == fqa.FQA_ERR_UNSUPPORTED

@@ -92,6 +92,33 @@ def test_tiled_core_identity_codec_is_exact_attention(bc):
     assert np.max(np.abs(out - ref)) < 1e-12
 
 
+@pytest.mark.parametrize("N,bc", [(200, 128), (77, 64), (129, 128), (1, 128)])
+def test_tiled_core_identity_codec_ragged_length(N, bc):
+    # N not a multiple of the tile (nor of the 64-token block): the last tile
+    # holds the remaining keys and the last block's scale covers the
+    # remaining tokens; unrounded, the rule is still exact softmax attention.
+    rng = np.random.default_rng(17)
+    d = 128
+    nb = (N + 63) // 64
+    qc, kc, vc = (rng.standard_normal((N, d)) * 3 for _ in range(3))
+    sq, sk, sv = (rng.uniform(0.2, 2.0, nb).astype(np.float32) for _ in range(3))
+    scale = 0.088
+    out = oracle.attention_core(qc, kc, vc, sq, sk, sv, float(sv.max()), scale, bc=bc, quantize_p=False)
+    rep = lambda a: np.repeat(a.astype(np.float64), 64)[:N, None]
+    ref = _scipy_attention(qc * rep(sq), kc * rep(sk), vc * rep(sv), scale)
+    assert np.max(np.abs(out - ref)) < 1e-12
+
+
+def test_exact_matches_scipy_ragged_length():
+    rng = np.random.default_rng(18)
+    N, d = 77, 128
+    q, k, v = (_bf16(rng.standard_normal((1, 1, N, d)) * 2) for _ in range(3))
+    sc = oracle.softmax_scale()
+    out = oracle.attention_exact(q, k, v, sc)[0]
+    qf, kf, vf = (s.bf16_bits_to_f32(t[0, 0]).astype(np.float64) for t in (q, k, v))
+    assert np.max(np.abs(out - _scipy_attention(qf, kf, vf, float(np.float32(sc))))) < 1e-12
+
+
 def test_rows_sum_to_one_identity_codec():
     rng = np.random.default_rng(8)
     N, d = 384, 128

@@ -86,7 +86,8 @@ def _reference_rows(qz, h, rows, scale, bc=128):
         m, l = None, Decimal(0)
         acc = [Decimal(0)] * d
         for t0 in range(0, N, bc):
-            xs = [Decimal(int(S[r, j])) * a_i * _dec(Fraction(float(sk[j // 64]))) for j in range(t0, t0 + bc)]
+            xs = [Decimal(int(S[r, j])) * a_i * _dec(Fraction(float(sk[j // 64])))
+                  for j in range(t0, min(t0 + bc, N))]
             m_new = max(xs) if m is None else max(m, max(xs))
             if m is not None:
                 alpha = ((m - m_new) * LN2).exp()
@@ -115,6 +116,22 @@ def test_oracle_fp8_matches_high_precision_reevaluation(h):
     rows = [0, 1, 63, 64, 130, 200, 255]
     ref = _reference_rows(qz, h, rows, scale)
     got, amb, _ = oracle.attention_fp8(qz, scale, heads=[(0, h)], rows=rows, with_ambiguity=True)
+    err = np.abs(got[0] - ref)
+    assert np.all(err <= 1e-10 * np.maximum(1.0, np.abs(ref)) + amb[0]), float(err.max())
+
+
+def test_oracle_fp8_ragged_length_matches_high_precision_reevaluation():
+    """N = 200: a short last 64-token block (8 tokens) and a short last KV tile
+    (72 keys); the re-evaluation runs the rule over the keys that exist."""
+    w = synth.workload("tiny_n256")
+    g = synth.generate(w)
+    q, k, v = (np.ascontiguousarray(g[t][:, :, :200]) for t in "qkv")
+    qz = oracle.quantize(q, k, v)
+    assert qz["sq"].shape == (1, 2, 4)
+    scale = oracle.softmax_scale()
+    rows = [0, 127, 128, 191, 192, 199]
+    ref = _reference_rows(qz, 1, rows, scale)
+    got, amb, _ = oracle.attention_fp8(qz, scale, heads=[(0, 1)], rows=rows, with_ambiguity=True)
     err = np.abs(got[0] - ref)
     assert np.all(err <= 1e-10 * np.maximum(1.0, np.abs(ref)) + amb[0]), float(err.max())
 

@@ -202,3 +202,47 @@ def test_smoothed_k_block_whose_scale_underflows_is_flushed():
     # no code anywhere is a NaN (S.1111.111)
     for name in ("q8", "k8", "v8"):
         assert not np.any((r[name] & 0x7F) == 0x7F)
+
+
+# ------------------------------------------------- sequences not a multiple of 64
+# [reading] the last block of a head holds the remaining N - 64*(nblk-1) tokens;
+# its scale is the absmax of those tokens alone; the K mean sums the short
+# block like the others and divides by N.
+
+def test_k_mean_short_last_block_exact_on_small_integers():
+    rng = np.random.default_rng(21)
+    k = rng.integers(-50, 50, size=(1, 2, 100, 128)).astype(np.float64)
+    mu = oracle.k_mean(_bf16(k)).astype(np.float64)
+    # every partial and total sum is an exact small integer, so only the final
+    # division rounds
+    assert np.array_equal(mu, (k.sum(axis=2) / 100.0).astype(np.float32).astype(np.float64))
+
+
+def test_k_mean_short_last_block_order_hand_case():
+    # N = 66: block 0 = 2^24 then 63 ones (each +1 is a tie back to 2^24), so
+    # p_0 = 2^24; block 1 has the 2 remaining tokens, 1 and 1: p_1 = 2;
+    # T = 2^24 + 2 (exact); mu = fl32((2^24 + 2) / 66).
+    k = np.zeros((1, 1, 66, 128))
+    k[0, 0, 0, 0] = 2.0 ** 24
+    k[0, 0, 1:66, 0] = 1.0
+    mu = oracle.k_mean(_bf16(k))
+    assert mu[0, 0, 0] == np.float32(np.float32(2.0 ** 24 + 2.0) / np.float32(66.0))
+
+
+def test_short_last_block_scale_is_its_own_absmax():
+    # N = 70: block 0 reaches |x| = 300, the 6-token block 1 only 3, so
+    # sq[1] = fl32(3/448) and its codes are E4M3(fl32(x * fl32(448/3))).
+    rng = np.random.default_rng(22)
+    x = rng.uniform(-2.5, 2.5, (1, 1, 70, 128))
+    x[0, 0, :64] *= 100.0
+    x[0, 0, 10, 3] = 300.0
+    x[0, 0, 66, 100] = -3.0
+    q = _bf16(x)
+    r = oracle.quantize(q, q, q)
+    assert r["sq"].shape == (1, 1, 2)
+    assert r["sq"][0, 0, 0] == np.float32(300.0) / np.float32(448.0)
+    assert r["sq"][0, 0, 1] == np.float32(3.0) / np.float32(448.0)
+    xf = s.bf16_bits_to_f32(q[0, 0, 64:]).astype(np.float32) * (np.float32(448.0) / np.float32(3.0))
+    ref = torch.from_numpy(xf).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(r["q8"][0, 0, 64:], ref)
+    assert r["sv_max"][0, 0] == r["sv"][0, 0, 0]
