@@ -69,6 +69,10 @@ def lib():
         L.orc_attention_fp8.argtypes = [P, P, P, P, P, P, P, i, i, i, i, ctypes.c_float, i,
                                         P, i, P, i, P, P, P]
         L.orc_attention_exact.argtypes = [P, P, P, i, i, i, i, ctypes.c_double, P, i, P, i, P]
+        L.orc_key_error.argtypes = [P, P, P, P, i, i, i, i, P]
+        L.orc_select_keys.argtypes = [P, i, i, i, i, P]
+        L.orc_attention_fp8_corrected.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, i, i, i, i,
+                                                  ctypes.c_float, i, P, i, P, i, P, P]
         L.orc_e4m3_encode_f32_array.argtypes = [P, ctypes.c_size_t, P]
         L.orc_bf16_round_array.argtypes = [P, ctypes.c_size_t, P]
         L.orc_num_threads.restype = i
@@ -197,6 +201,51 @@ def attention_core(qc, kc, vc, sq, sk, sv, sv_max, scale, bc=128, quantize_p=Tru
                              _p(out), None if amb is None else _p(amb),
                              None if namb is None else _p(namb))
     return (out, amb, namb) if with_ambiguity else out
+
+
+# ------------------------------------------------ error-corrected attention
+
+def key_error(k_bf16: np.ndarray, qz: dict) -> np.ndarray:
+    """Per-key quantization error [B,H,N] (binary32, pinned order; see the C file)."""
+    B, H, N, d = k_bf16.shape
+    k_bf16 = np.ascontiguousarray(k_bf16, dtype=np.uint16)
+    err = np.empty((B, H, N), dtype=np.float32)
+    lib().orc_key_error(_p(k_bf16), _p(qz["k8"]), _p(qz["sk"]), _p(qz["k_mean"]), B, H, N, d, _p(err))
+    return err
+
+
+def n_corrected(N: int, rho: float) -> int:
+    """Keys corrected per head: ceil(rho * N), clamped to [0, N]."""
+    import math
+    return max(0, min(N, math.ceil(float(rho) * N - 1e-9)))
+
+
+def select_keys(err: np.ndarray, kc: int) -> np.ndarray:
+    """[B,H,N] 0/1: the kc keys of each head with the largest error (ties to the
+    lower index)."""
+    B, H, N = err.shape
+    err = np.ascontiguousarray(err, dtype=np.float32)
+    sel = np.empty((B, H, N), dtype=np.uint8)
+    lib().orc_select_keys(_p(err), B, H, N, int(kc), _p(sel))
+    return sel
+
+
+def attention_fp8_corrected(g: dict, qz: dict, sel: np.ndarray, softmax_scale: float, heads=None,
+                            rows=None, quantize_p: bool = True, with_ambiguity: bool = False):
+    """Error-corrected FP8 attention -> [n_heads, n_rows, d] binary64 (and the
+    ambiguity bound of its FP8 part when with_ambiguity)."""
+    B, H, N, d = qz["q8"].shape
+    ha, ra = _heads_rows(B, H, N, heads, rows)
+    out = np.empty((len(ha), len(ra), d), dtype=np.float64)
+    amb = np.empty_like(out) if with_ambiguity else None
+    q, k, v = (np.ascontiguousarray(g[t], dtype=np.uint16) for t in "qkv")
+    sel = np.ascontiguousarray(sel, dtype=np.uint8)
+    lib().orc_attention_fp8_corrected(
+        _p(q), _p(k), _p(v), _p(qz["q8"]), _p(qz["k8"]), _p(qz["v8"]), _p(qz["sq"]), _p(qz["sk"]),
+        _p(qz["sv"]), _p(qz["sv_max"]), _p(qz["k_mean"]), _p(sel), B, H, N, d,
+        float(np.float32(softmax_scale)), int(bool(quantize_p)), _p(ha), len(ha), _p(ra), len(ra),
+        _p(out), None if amb is None else _p(amb))
+    return (out, amb) if with_ambiguity else out
 
 
 def attention_exact(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float,

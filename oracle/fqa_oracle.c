@@ -248,11 +248,17 @@ static double p_eval_bound(double abs_prod_sum, double a, double x, double m)
     return LN2 * dx + ldexp(1.0, -21) + ldexp(1.0, -22);
 }
 
+/* skip (optional, [N]): keys with skip[j] != 0 take no part in the rule (no
+ * maximum, p, row-sum term or P code) -- the keys an error-corrected pass
+ * handles exactly; a tile with none left changes nothing.  m_out, l_out
+ * (optional, [n_rows]): the final running maximum and row sum (l = 0 when
+ * every key is skipped; the output row is then 0). */
 static void attention_core_head(const double *qc, const double *kc, const double *vc,
                                 const float *sq, const float *sk, const float *sv, float sv_max,
                                 int N, int d, double scale, int bc, int quantize_p,
                                 const int *rows, int n_rows, double *out,
-                                double *amb, int *namb)
+                                double *amb, int *namb, const uint8_t *skip,
+                                double *m_out, double *l_out)
 {
     const double LOG2E = 1.4426950408889634073599246810019;  /* log2(e) */
     #pragma omp parallel for schedule(dynamic, 4)
@@ -269,6 +275,8 @@ static void attention_core_head(const double *qc, const double *kc, const double
             for (int c = 0; c < d; c++) o[c] = 0.0;
             if (amb) for (int c = 0; c < d; c++) amb[(size_t)r * d + c] = 0.0;
             if (namb) namb[r] = 0;
+            if (m_out) m_out[r] = 0.0;           /* V is all zero: any weight gives 0 */
+            if (l_out) l_out[r] = 1.0;
             free(x); free(aps); free(acc); free(aacc);
             continue;
         }
@@ -277,6 +285,11 @@ static void attention_core_head(const double *qc, const double *kc, const double
             double tmax = -INFINITY;
             for (int j = t0; j < t1; j++) {
                 double s = 0.0, sa = 0.0;
+                if (skip && skip[j]) {
+                    x[j - t0] = -INFINITY;
+                    aps[j - t0] = 0.0;
+                    continue;
+                }
                 for (int c = 0; c < d; c++) {
                     double pr = qc[(size_t)i * d + c] * kc[(size_t)j * d + c];
                     s += pr;
@@ -287,11 +300,15 @@ static void attention_core_head(const double *qc, const double *kc, const double
                 if (x[j - t0] > tmax) tmax = x[j - t0];
             }
             double m_new = tmax > m ? tmax : m;
+            if (m_new == -INFINITY)              /* no key yet: nothing to do */
+                continue;
             double alpha = exp2(m - m_new);      /* 0 on the first tile */
             l *= alpha;
             for (int c = 0; c < d; c++) acc[c] *= alpha;
             for (int c = 0; c < d; c++) aacc[c] *= alpha;
             for (int j = t0; j < t1; j++) {
+                if (skip && skip[j])
+                    continue;
                 double p = exp2(x[j - t0] - m_new);
                 double rv = (double)sv[j / 64] / (double)sv_max;
                 double P = p * 448.0 * rv;
@@ -322,11 +339,13 @@ static void attention_core_head(const double *qc, const double *kc, const double
             m = m_new;
         }
         for (int c = 0; c < d; c++)
-            o[c] = acc[c] * ((double)sv_max / 448.0) / l;
+            o[c] = l > 0.0 ? acc[c] * ((double)sv_max / 448.0) / l : 0.0;
         if (amb)
             for (int c = 0; c < d; c++)
-                amb[(size_t)r * d + c] = aacc[c] * ((double)sv_max / 448.0) / l;
+                amb[(size_t)r * d + c] = l > 0.0 ? aacc[c] * ((double)sv_max / 448.0) / l : 0.0;
         if (namb) namb[r] = n_amb;
+        if (m_out) m_out[r] = m;
+        if (l_out) l_out[r] = l;
         free(x);
         free(aps);
         free(acc);
@@ -341,7 +360,7 @@ void orc_attention_core(const double *qc, const double *kc, const double *vc,
                         const int *rows, int n_rows, double *out, double *amb, int *namb)
 {
     attention_core_head(qc, kc, vc, sq, sk, sv, sv_max, N, d, scale, bc, quantize_p,
-                        rows, n_rows, out, amb, namb);
+                        rows, n_rows, out, amb, namb, NULL, NULL, NULL);
 }
 
 /* FP8 attention on quantizer outputs (codes in natural [B,H,N,d] layout).
@@ -373,9 +392,178 @@ void orc_attention_fp8(const uint8_t *q8, const uint8_t *k8, const uint8_t *v8,
                             sv_max[(size_t)b * H + h], N, d, (double)softmax_scale, bc, 1,
                             rows, n_rows, out + (size_t)hh * n_rows * d,
                             amb ? amb + (size_t)hh * n_rows * d : NULL,
-                            namb ? namb + (size_t)hh * n_rows : NULL);
+                            namb ? namb + (size_t)hh * n_rows : NULL, NULL, NULL, NULL);
     }
     free(qc); free(kc); free(vc);
+}
+
+/* --------------------------------------------- error-corrected attention */
+/* FP8 attention that corrects only the tokens with large error: "FLUX 3
+ * Image Klein Base: 생성 3.46배, 8장 확장 병목", section "왜 이런 차이가 나나"
+ * (VC-Attention FP8, rho = 0.005, against cuDNN FP8 and VANILLA BF16 on
+ * B200).  The page gives the name, the idea and rho only; the readings:
+ *  - the tokens are key/value tokens and the error is each key's own
+ *    quantization error (orc_key_error);
+ *  - per (b, h) the ceil(rho * N) keys with the largest error are corrected
+ *    (orc_select_keys);
+ *  - correction: the FP8 rule runs over the other keys, the corrected keys'
+ *    part is exact (binary64 from the BF16 inputs, scores on the smoothed
+ *    keys so both parts share one per-row offset), and the two partial
+ *    softmaxes are merged by their maxima and row sums. */
+
+/* Per-key quantization error [reading]: the squared distance between the
+ * smoothed key and its dequantized code, in binary32 in a pinned order:
+ *   r_c = fl32(x_c - fl32(dec(code_c) * s_J)),  x_c = fl32(k_c - mu_c)
+ *   g_i = ((r_8i^2 + r_8i+1^2) + ...) + r_8i+7^2   (i = 0..15, squares rounded)
+ *   then pairwise: a_i = g_i + g_i+8, b_i = a_i + a_i+4, c_i = b_i + b_i+2,
+ *   e = c_0 + c_1.
+ * err: [B,H,N]. */
+void orc_key_error(const uint16_t *k, const uint8_t *k8, const float *sk, const float *k_mean,
+                   int B, int H, int N, int d, float *err)
+{
+    int nblk = (N + 63) / 64;
+    float dec[256];
+    for (int i = 0; i < 256; i++) dec[i] = (float)orc_e4m3_decode((uint8_t)i);
+    #pragma omp parallel for collapse(2) schedule(static)
+    for (int b = 0; b < B; b++)
+        for (int h = 0; h < H; h++) {
+            const float *mu = k_mean + ((size_t)b * H + h) * d;
+            for (int n = 0; n < N; n++) {
+                float s = sk[((size_t)b * H + h) * nblk + n / 64];
+                float g[16];
+                for (int i = 0; i < 16; i++) {
+                    float acc = 0.0f;
+                    for (int c = 8 * i; c < 8 * i + 8; c++) {
+                        size_t at = IDX4(b, h, n, c, H, N, d);
+                        float x = orc_bf16_to_float(k[at]) - mu[c];
+                        float dq = dec[k8[at]] * s;
+                        float rr = x - dq;
+                        float sq = rr * rr;
+                        acc = acc + sq;
+                    }
+                    g[i] = acc;
+                }
+                float a[8], bb[4], cc[2];
+                for (int i = 0; i < 8; i++) a[i] = g[i] + g[i + 8];
+                for (int i = 0; i < 4; i++) bb[i] = a[i] + a[i + 4];
+                for (int i = 0; i < 2; i++) cc[i] = bb[i] + bb[i + 2];
+                err[((size_t)b * H + h) * N + n] = cc[0] + cc[1];
+            }
+        }
+}
+
+/* The kc keys of each (b, h) with the largest error, ties to the lower token
+ * index: sel[B,H,N] = 1 for them, 0 otherwise (kc is clamped to [0, N]). */
+static const float *g_sel_err;
+static int sel_cmp(const void *pa, const void *pb)
+{
+    int ia = *(const int *)pa, ib = *(const int *)pb;
+    float ea = g_sel_err[ia], eb = g_sel_err[ib];
+    if (ea > eb) return -1;
+    if (ea < eb) return 1;
+    return ia < ib ? -1 : (ia > ib ? 1 : 0);
+}
+
+void orc_select_keys(const float *err, int B, int H, int N, int kc, uint8_t *sel)
+{
+    if (kc < 0) kc = 0;
+    if (kc > N) kc = N;
+    int *idx = (int *)malloc(sizeof(int) * N);
+    for (int bh = 0; bh < B * H; bh++) {
+        const float *e = err + (size_t)bh * N;
+        for (int j = 0; j < N; j++) idx[j] = j;
+        g_sel_err = e;                          /* single-threaded: qsort has no context */
+        qsort(idx, N, sizeof(int), sel_cmp);
+        memset(sel + (size_t)bh * N, 0, N);
+        for (int t = 0; t < kc; t++) sel[(size_t)bh * N + idx[t]] = 1;
+    }
+    free(idx);
+}
+
+/* Error-corrected FP8 attention for the listed heads and rows.  q, k, v: the
+ * BF16 inputs; the code/scale arrays and k_mean from orc_quantize; sel from
+ * orc_select_keys.  For row i:
+ *   FP8 part over keys with sel = 0 (the tiled rule): O1, m1, l1
+ *   exact part over keys with sel = 1: s_j = (q_i . (k_j - mu)) * scale * log2(e),
+ *     m2 = max s_j, p_j = 2^(s_j - m2), l2 = sum p_j, A2 = sum p_j v_j
+ *   M = max(m1, m2), w1 = 2^(m1 - M), w2 = 2^(m2 - M) (0 for an empty part),
+ *   out = (O1 * l1 * w1 + A2 * w2) / (l1 * w1 + l2 * w2).
+ * quantize_p = 0 leaves the FP8 part's P unrounded (for the pins).  amb
+ * (optional): the FP8 part's ambiguity bound, carried through the merge. */
+void orc_attention_fp8_corrected(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                                 const uint8_t *q8, const uint8_t *k8, const uint8_t *v8,
+                                 const float *sq, const float *sk, const float *sv,
+                                 const float *sv_max, const float *k_mean, const uint8_t *sel,
+                                 int B, int H, int N, int d, float softmax_scale, int quantize_p,
+                                 const int *heads, int n_heads, const int *rows, int n_rows,
+                                 double *out, double *amb)
+{
+    const double LOG2E = 1.4426950408889634073599246810019;
+    int nblk = (N + 63) / 64;
+    (void)B;
+    double *qc = (double *)malloc(sizeof(double) * N * d);
+    double *kc = (double *)malloc(sizeof(double) * N * d);
+    double *vc = (double *)malloc(sizeof(double) * N * d);
+    double *m1 = (double *)malloc(sizeof(double) * n_rows);
+    double *l1 = (double *)malloc(sizeof(double) * n_rows);
+    double dec[256];
+    for (int i = 0; i < 256; i++) dec[i] = orc_e4m3_decode((uint8_t)i);
+    for (int hh = 0; hh < n_heads; hh++) {
+        int b = heads[2 * hh], h = heads[2 * hh + 1];
+        size_t base = IDX4(b, h, 0, 0, H, N, d);
+        const uint8_t *sl = sel + ((size_t)b * H + h) * N;
+        const float *mu = k_mean + ((size_t)b * H + h) * d;
+        for (size_t i = 0; i < (size_t)N * d; i++) {
+            qc[i] = dec[q8[base + i]];
+            kc[i] = dec[k8[base + i]];
+            vc[i] = dec[v8[base + i]];
+        }
+        size_t sidx = ((size_t)b * H + h) * nblk;
+        double *o = out + (size_t)hh * n_rows * d;
+        double *ab = amb ? amb + (size_t)hh * n_rows * d : NULL;
+        attention_core_head(qc, kc, vc, sq + sidx, sk + sidx, sv + sidx,
+                            sv_max[(size_t)b * H + h], N, d, (double)softmax_scale, 128,
+                            quantize_p, rows, n_rows, o, ab, NULL, sl, m1, l1);
+        #pragma omp parallel for schedule(dynamic, 4)
+        for (int r = 0; r < n_rows; r++) {
+            int i = rows[r];
+            double qi[512];
+            for (int c = 0; c < d && c < 512; c++)
+                qi[c] = orc_bf16_to_float(q[base + (size_t)i * d + c]);
+            double m2 = -INFINITY;
+            for (int j = 0; j < N; j++) {
+                if (!sl[j]) continue;
+                double s = 0.0;
+                for (int c = 0; c < d; c++)
+                    s += qi[c] * ((double)orc_bf16_to_float(k[base + (size_t)j * d + c]) - (double)mu[c]);
+                s *= (double)softmax_scale * LOG2E;
+                if (s > m2) m2 = s;
+            }
+            double l2 = 0.0, a2[512];
+            for (int c = 0; c < d; c++) a2[c] = 0.0;
+            if (m2 > -INFINITY)
+                for (int j = 0; j < N; j++) {
+                    if (!sl[j]) continue;
+                    double s = 0.0;
+                    for (int c = 0; c < d; c++)
+                        s += qi[c] * ((double)orc_bf16_to_float(k[base + (size_t)j * d + c]) - (double)mu[c]);
+                    double p = exp2(s * (double)softmax_scale * LOG2E - m2);
+                    l2 += p;
+                    for (int c = 0; c < d; c++)
+                        a2[c] += p * orc_bf16_to_float(v[base + (size_t)j * d + c]);
+                }
+            double mm = m1[r] > m2 ? m1[r] : m2;
+            double w1 = (l1[r] > 0.0) ? exp2(m1[r] - mm) : 0.0;
+            double w2 = (m2 > -INFINITY) ? exp2(m2 - mm) : 0.0;
+            double L = l1[r] * w1 + l2 * w2;
+            for (int c = 0; c < d; c++) {
+                double v1 = o[(size_t)r * d + c] * l1[r] * w1;
+                o[(size_t)r * d + c] = L > 0.0 ? (v1 + a2[c] * w2) / L : 0.0;
+                if (ab) ab[(size_t)r * d + c] = L > 0.0 ? ab[(size_t)r * d + c] * l1[r] * w1 / L : 0.0;
+            }
+        }
+    }
+    free(qc); free(kc); free(vc); free(m1); free(l1);
 }
 
 /* Exact attention, binary64, no quantization: softmax(Q K^T * scale) V on the
