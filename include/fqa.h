@@ -134,6 +134,24 @@ FQA_API fqa_status fqa_quantize(const void* q, const void* k, const void* v, int
                         void* cuda_stream);
 
 /*
+ * fqa_quantize_keyerr -- fqa_quantize() that also writes each key's
+ * quantization error, the selection metric of fqa_attention_fp8_corrected().
+ * [KLEIN] section "왜 이런 차이가 나나" (VC-Attention FP8 corrects the tokens
+ * with large error); the error measure is a reading:
+ *   k_err[b,h,n] = sum over channels c of r_c^2, r_c = fl32(x_c - fl32(dec(k8_c) * sk)),
+ *   x_c = fl32(k_c - k_mean[c]), each square rounded to binary32, summed in a
+ *   pinned order: 16 groups of 8 consecutive channels summed sequentially,
+ *   then g_i + g_i+8, then + the term 4 apart, 2 apart, 1 apart.
+ * Same arguments and results as fqa_quantize() plus
+ * k_err  out: FP32 [B,H,N] (4-byte aligned, not NULL).
+ * Computed in the same launch (no extra pass over K).
+ */
+FQA_API fqa_status fqa_quantize_keyerr(const void* q, const void* k, const void* v, int B, int H, int N,
+                                       int d, void* q8, void* k8, void* v8, float* sq, float* sk,
+                                       float* sv, float* sv_max, float* k_mean, float* k_err,
+                                       void* workspace, size_t workspace_bytes, void* cuda_stream);
+
+/*
  * fqa_quantize_noalloc -- fqa_quantize() without a workspace argument, for
  * callers that cannot allocate device memory at call time: for example an
  * operator running inside a host framework that owns all device memory and
@@ -209,6 +227,65 @@ FQA_API fqa_status fqa_attention_fp8(const void* q8, const void* k8, const void*
 FQA_API fqa_status fqa_attention_bf16(const void* q, const void* k, const void* v, int B, int H, int N,
                               int d, float softmax_scale, void* out, fqa_out_dtype out_dtype,
                               void* cuda_stream);
+
+/*
+ * Error-corrected FP8 attention: FP8 attention that corrects only the tokens
+ * with large error.  [KLEIN] section "왜 이런 차이가 나나": VC-Attention FP8
+ * (rho = 0.005) is one of the B200 FP8 attention backends measured there; the
+ * page gives the name, the idea and rho only.  Readings: the corrected tokens
+ * are, per (b, h), the fqa_corrected_keys(N, rho) keys with the largest
+ * k_err (ties to the lower index); their part of the softmax is computed
+ * exactly from the BF16 inputs (scores on the smoothed keys,
+ * (q . k - q . k_mean) * softmax_scale), the FP8 rule of fqa_attention_fp8()
+ * runs over the other keys, and the two partial softmaxes are merged by their
+ * maxima and row sums.
+ */
+
+/* Keys corrected per head: ceil(rho * N - 0.01) clamped to [0, N] (rho is
+ * binary32, whose rounding moves rho * N by at most 0.004 for N <= 65536: a
+ * product meant to be an integer stays that integer); -1 for N < 1 or rho
+ * outside [0, 1]. */
+FQA_API int fqa_corrected_keys(int N, float rho);
+
+/*
+ * fqa_select_keys -- the kc keys of each (b, h) with the largest k_err, ties
+ * to the lower token index.  k_err: FP32 [B,H,N] (fqa_quantize_keyerr);
+ * kmask out: uint32 [B,H,ceil(N/32)], bit k of word w set when key 32w + k
+ * is selected; idx out: int32 [B,H,kc], the selected keys in ascending order.
+ * 1 <= kc <= N.  One launch, one CTA per (b, h).
+ */
+FQA_API fqa_status fqa_select_keys(const float* k_err, int B, int H, int N, int kc, uint32_t* kmask,
+                                   int* idx, void* cuda_stream);
+
+/* Workspace bytes of fqa_attention_fp8_corrected(): the key mask, the
+ * corrected indices, each row's FP8-part (m, l) and the FP8 part's FP32
+ * output (B*H*N*512 bytes dominate); 0 for invalid sizes. */
+FQA_API size_t fqa_attention_fp8_corrected_workspace_bytes(int B, int H, int N, int d, float rho);
+
+/*
+ * fqa_attention_fp8_corrected -- error-corrected FP8 attention.
+ * q, k, v: the BF16 inputs [B,H,N,d]; q8 .. k_mean: the fqa_quantize_keyerr()
+ * outputs for them; k_err: its key errors; rho in [0, 1] (0 = plain FP8
+ * attention); out: [B,H,N,d] BF16 or FP32; workspace of at least
+ * fqa_attention_fp8_corrected_workspace_bytes(), 16-byte aligned.
+ * For query row i, with C the selected keys of its head:
+ *   FP8 part over keys not in C (the fqa_attention_fp8() rule, keys in C
+ *   taking no part): normalized output O1, maximum m1, row sum l1;
+ *   exact part over C: s_j = (q_i . k_j - q_i . k_mean) * softmax_scale * log2(e),
+ *   m2 = max s_j, p_j = 2^(s_j - m2), l2 = sum p_j, A2 = sum p_j v_j;
+ *   out_i = (O1 l1 2^(m1 - M) + A2 2^(m2 - M)) / (l1 2^(m1 - M) + l2 2^(m2 - M)),
+ *   M = max(m1, m2).
+ * The exact part runs in FP32 on the tensor cores (BF16 operands, P split
+ * into BF16 high and low parts).  Enqueues the selection, the FP8 attention
+ * launch with the key mask, and the exact part and merge.
+ */
+FQA_API fqa_status fqa_attention_fp8_corrected(const void* q, const void* k, const void* v, const void* q8,
+                                               const void* k8, const void* v8, const float* sq,
+                                               const float* sk, const float* sv, const float* sv_max,
+                                               const float* k_mean, const float* k_err, int B, int H, int N,
+                                               int d, float softmax_scale, float rho, void* out,
+                                               fqa_out_dtype out_dtype, void* workspace,
+                                               size_t workspace_bytes, void* cuda_stream);
 
 /*
  * fqa_e4m3_encode -- the library's binary32 -> E4M3 conversion (round to

@@ -73,6 +73,8 @@ def lib():
         L.orc_select_keys.argtypes = [P, i, i, i, i, P]
         L.orc_attention_fp8_corrected.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, i, i, i, i,
                                                   ctypes.c_float, i, P, i, P, i, P, P]
+        L.orc_attention_fp8_part.argtypes = [P, P, P, P, P, P, P, P, i, i, i, i, ctypes.c_float, P, i, P, i,
+                                             P, P, P]
         L.orc_e4m3_encode_f32_array.argtypes = [P, ctypes.c_size_t, P]
         L.orc_bf16_round_array.argtypes = [P, ctypes.c_size_t, P]
         L.orc_num_threads.restype = i
@@ -215,9 +217,11 @@ def key_error(k_bf16: np.ndarray, qz: dict) -> np.ndarray:
 
 
 def n_corrected(N: int, rho: float) -> int:
-    """Keys corrected per head: ceil(rho * N), clamped to [0, N]."""
+    """Keys corrected per head [reading]: ceil(fl32(rho) * N - 0.01), clamped to
+    [0, N] -- rho in binary32 as the C ABI takes it; the 0.01 keeps a product
+    meant to be an integer (0.05 of 1280 keys) that integer."""
     import math
-    return max(0, min(N, math.ceil(float(rho) * N - 1e-9)))
+    return max(0, min(N, math.ceil(float(np.float32(rho)) * N - 0.01)))
 
 
 def select_keys(err: np.ndarray, kc: int) -> np.ndarray:
@@ -228,6 +232,22 @@ def select_keys(err: np.ndarray, kc: int) -> np.ndarray:
     sel = np.empty((B, H, N), dtype=np.uint8)
     lib().orc_select_keys(_p(err), B, H, N, int(kc), _p(sel))
     return sel
+
+
+def attention_fp8_part(qz: dict, sel: np.ndarray, softmax_scale: float, heads=None, rows=None):
+    """The FP8 rule over the keys with sel = 0 -> (out [n_heads, n_rows, d],
+    m [n_heads, n_rows], l [n_heads, n_rows]) in binary64."""
+    B, H, N, d = qz["q8"].shape
+    ha, ra = _heads_rows(B, H, N, heads, rows)
+    out = np.empty((len(ha), len(ra), d), dtype=np.float64)
+    m = np.empty((len(ha), len(ra)), dtype=np.float64)
+    l = np.empty_like(m)
+    sel = np.ascontiguousarray(sel, dtype=np.uint8)
+    lib().orc_attention_fp8_part(_p(qz["q8"]), _p(qz["k8"]), _p(qz["v8"]), _p(qz["sq"]), _p(qz["sk"]),
+                                 _p(qz["sv"]), _p(qz["sv_max"]), _p(sel), B, H, N, d,
+                                 float(np.float32(softmax_scale)), _p(ha), len(ha), _p(ra), len(ra), _p(out),
+                                 _p(m), _p(l))
+    return out, m, l
 
 
 def attention_fp8_corrected(g: dict, qz: dict, sel: np.ndarray, softmax_scale: float, heads=None,

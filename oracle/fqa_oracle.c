@@ -480,6 +480,40 @@ void orc_select_keys(const float *err, int B, int H, int N, int kc, uint8_t *sel
     free(idx);
 }
 
+/* The FP8 part alone: the tiled rule over the keys with sel = 0 (normalized
+ * output, and each row's final maximum and row sum; l = 0 and a zero row
+ * when every key is selected).  out: [n_heads, n_rows, d]; m_out, l_out:
+ * [n_heads, n_rows]. */
+void orc_attention_fp8_part(const uint8_t *q8, const uint8_t *k8, const uint8_t *v8,
+                            const float *sq, const float *sk, const float *sv, const float *sv_max,
+                            const uint8_t *sel, int B, int H, int N, int d, float softmax_scale,
+                            const int *heads, int n_heads, const int *rows, int n_rows,
+                            double *out, double *m_out, double *l_out)
+{
+    int nblk = (N + 63) / 64;
+    (void)B;
+    double *qc = (double *)malloc(sizeof(double) * N * d);
+    double *kc = (double *)malloc(sizeof(double) * N * d);
+    double *vc = (double *)malloc(sizeof(double) * N * d);
+    double dec[256];
+    for (int i = 0; i < 256; i++) dec[i] = orc_e4m3_decode((uint8_t)i);
+    for (int hh = 0; hh < n_heads; hh++) {
+        int b = heads[2 * hh], h = heads[2 * hh + 1];
+        size_t base = IDX4(b, h, 0, 0, H, N, d);
+        for (size_t i = 0; i < (size_t)N * d; i++) {
+            qc[i] = dec[q8[base + i]];
+            kc[i] = dec[k8[base + i]];
+            vc[i] = dec[v8[base + i]];
+        }
+        size_t sidx = ((size_t)b * H + h) * nblk;
+        attention_core_head(qc, kc, vc, sq + sidx, sk + sidx, sv + sidx, sv_max[(size_t)b * H + h], N, d,
+                            (double)softmax_scale, 128, 1, rows, n_rows, out + (size_t)hh * n_rows * d,
+                            NULL, NULL, sel + ((size_t)b * H + h) * N, m_out + (size_t)hh * n_rows,
+                            l_out + (size_t)hh * n_rows);
+    }
+    free(qc); free(kc); free(vc);
+}
+
 /* Error-corrected FP8 attention for the listed heads and rows.  q, k, v: the
  * BF16 inputs; the code/scale arrays and k_mean from orc_quantize; sel from
  * orc_select_keys.  For row i:

@@ -54,6 +54,17 @@ def _load():
     L.fqa_e4m3_encode.argtypes = [P, P, ctypes.c_size_t, P]
     L.fqa_debug_status.restype = I
     L.fqa_debug_status.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
+    L.fqa_quantize_keyerr.restype = I
+    L.fqa_quantize_keyerr.argtypes = [P, P, P, I, I, I, I, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+    L.fqa_corrected_keys.restype = I
+    L.fqa_corrected_keys.argtypes = [I, ctypes.c_float]
+    L.fqa_select_keys.restype = I
+    L.fqa_select_keys.argtypes = [P, I, I, I, I, P, P, P]
+    L.fqa_attention_fp8_corrected_workspace_bytes.restype = ctypes.c_size_t
+    L.fqa_attention_fp8_corrected_workspace_bytes.argtypes = [I, I, I, I, ctypes.c_float]
+    L.fqa_attention_fp8_corrected.restype = I
+    L.fqa_attention_fp8_corrected.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, I, I, I, I, ctypes.c_float,
+                                              ctypes.c_float, P, I, P, ctypes.c_size_t, P]
     _lib = L
     return L
 
@@ -132,6 +143,38 @@ def fqa_attention_bf16(q, k, v, softmax_scale, out, out_dtype, stream=None) -> i
     B, H, N, d = q.shape
     return _load().fqa_attention_bf16(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, float(softmax_scale),
                                    _ptr(out), int(out_dtype), _stream(stream))
+
+
+def fqa_quantize_keyerr(q, k, v, q8, k8, v8, sq, sk, sv, sv_max, k_mean, k_err, workspace,
+                        stream=None) -> int:
+    """fqa_quantize plus each key's quantization error k_err [B,H,N] FP32."""
+    B, H, N, d = q.shape
+    return _load().fqa_quantize_keyerr(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, _ptr(q8), _ptr(k8), _ptr(v8),
+                                    _ptr(sq), _ptr(sk), _ptr(sv), _ptr(sv_max), _ptr(k_mean), _ptr(k_err),
+                                    _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                    _stream(stream))
+
+
+def fqa_corrected_keys(N: int, rho: float) -> int:
+    return int(_load().fqa_corrected_keys(int(N), float(rho)))
+
+
+def fqa_select_keys(k_err, kc: int, kmask, idx, stream=None) -> int:
+    B, H, N = k_err.shape
+    return _load().fqa_select_keys(_ptr(k_err), B, H, N, int(kc), _ptr(kmask), _ptr(idx), _stream(stream))
+
+
+def fqa_attention_fp8_corrected_workspace_bytes(B: int, H: int, N: int, rho: float, d: int = HEAD_DIM) -> int:
+    return int(_load().fqa_attention_fp8_corrected_workspace_bytes(B, H, N, d, float(rho)))
+
+
+def fqa_attention_fp8_corrected(q, k, v, q8, k8, v8, sq, sk, sv, sv_max, k_mean, k_err, softmax_scale, rho,
+                                out, out_dtype, workspace, stream=None) -> int:
+    B, H, N, d = q.shape
+    return _load().fqa_attention_fp8_corrected(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(q8), _ptr(k8), _ptr(v8), _ptr(sq), _ptr(sk), _ptr(sv), _ptr(sv_max),
+        _ptr(k_mean), _ptr(k_err), B, H, N, d, float(softmax_scale), float(rho), _ptr(out), int(out_dtype),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
 
 
 def fqa_e4m3_encode(x, out, stream=None) -> int:
@@ -258,6 +301,52 @@ def attention_bf16(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, softmax_sc
     _require(out, dt, "out", (B, H, N, d))
     _check(fqa_attention_bf16(q, k, v, softmax_scale, out, out_dtype, stream=stream),
            "fqa_attention_bf16")
+    return out
+
+
+def quantize_keyerr(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: Optional[Quantized] = None,
+                    k_err: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                    stream=None):
+    """quantize() plus the per-key quantization error: (Quantized, k_err [B,H,N] float32)."""
+    B, H, N, _ = _require_qkv(q, k, v, torch.bfloat16)
+    if out is None:
+        out = alloc_quantized(B, H, N, q.device)
+    _require_quantized(out, B, H, N)
+    if k_err is None:
+        k_err = torch.empty(B, H, N, dtype=torch.float32, device=q.device)
+    _require(k_err, torch.float32, "k_err", (B, H, N))
+    if workspace is None:
+        workspace = alloc_workspace(B, H, N, q.device)
+    _require(workspace, workspace.dtype, "workspace")
+    _check(fqa_quantize_keyerr(q, k, v, *out, k_err, workspace, stream=stream), "fqa_quantize_keyerr")
+    return out, k_err
+
+
+def alloc_corrected_workspace(B: int, H: int, N: int, rho: float, device) -> torch.Tensor:
+    nbytes = fqa_attention_fp8_corrected_workspace_bytes(B, H, N, rho)
+    if nbytes == 0:
+        raise ValueError("invalid sizes or rho for the corrected path")
+    return torch.empty((nbytes + 15) // 16 * 4, dtype=torch.float32, device=device)
+
+
+def attention_fp8_corrected(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, qz: Quantized,
+                            k_err: torch.Tensor, softmax_scale: float, rho: float = 0.005,
+                            out_dtype: int = FQA_OUT_BF16, out: Optional[torch.Tensor] = None,
+                            workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Error-corrected FP8 attention: the ceil(rho * N) keys per head with the
+    largest quantization error are handled exactly, the rest by the FP8 rule."""
+    B, H, N, d = _require_qkv(q, k, v, torch.bfloat16)
+    _require_quantized(qz, B, H, N)
+    _require(k_err, torch.float32, "k_err", (B, H, N))
+    dt = torch.float32 if out_dtype == FQA_OUT_F32 else torch.bfloat16
+    if out is None:
+        out = torch.empty(B, H, N, d, dtype=dt, device=q.device)
+    _require(out, dt, "out", (B, H, N, d))
+    if workspace is None:
+        workspace = alloc_corrected_workspace(B, H, N, rho, q.device)
+    _require(workspace, workspace.dtype, "workspace")
+    _check(fqa_attention_fp8_corrected(q, k, v, *qz[:7], qz.k_mean, k_err, softmax_scale, rho, out, out_dtype,
+                                       workspace, stream=stream), "fqa_attention_fp8_corrected")
     return out
 
 

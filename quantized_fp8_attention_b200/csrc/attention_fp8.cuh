@@ -441,7 +441,9 @@ __global__ void __launch_bounds__(kF8Threads, 1)
         // a tile with no key present, after tiles with none, leaves
         // m = m_new = -inf with nothing to rescale (key masks only)
         const float alpha = (kMaskable && m_new == -INFINITY) ? 1.0f : ex2_approx(m - m_new);
-        const float2 nm2 = make_float2(-m_new, -m_new);
+        // (and -inf - -inf would be NaN: with no key present, subtract 0)
+        const float nm = (kMaskable && m_new == -INFINITY) ? 0.0f : -m_new;
+        const float2 nm2 = make_float2(nm, nm);
         const float2 a2 = make_float2(ah, ah);
         float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
         const uint32_t pbuf = prow + (uint32_t)(g & 1) * T::kTileBytes;

@@ -13,6 +13,7 @@
 #include "attention.cuh"
 #include "attention_fp8.cuh"
 #include "attention_ws.cuh"
+#include "correct.cuh"
 #include "device.cuh"
 #include "quantize.cuh"
 
@@ -196,10 +197,10 @@ size_t fqa_quantize_workspace_bytes(int B, int H, int N, int d) {
   return ((partial_bytes(B, H, N, d) + 255) & ~size_t(255)) + 256;
 }
 
-fqa_status fqa_quantize(const void* q, const void* k, const void* v, int B, int H, int N, int d,
-                        void* q8, void* k8, void* v8, float* sq, float* sk, float* sv,
-                        float* sv_max, float* k_mean, void* workspace, size_t workspace_bytes,
-                        void* cuda_stream) {
+static fqa_status quantize_impl(const void* q, const void* k, const void* v, int B, int H, int N, int d,
+                                void* q8, void* k8, void* v8, float* sq, float* sk, float* sv,
+                                float* sv_max, float* k_mean, float* k_err, void* workspace,
+                                size_t workspace_bytes, void* cuda_stream) {
   fqa_status st = check_shape(B, H, N, d);
   if (st != FQA_OK) return st;
   const void* ptrs[] = {q, k, v, q8, k8, v8, sq, sk, sv, sv_max, k_mean, workspace};
@@ -209,7 +210,7 @@ fqa_status fqa_quantize(const void* q, const void* k, const void* v, int B, int 
   const void* a16[] = {q, k, v, q8, k8, v8, k_mean, workspace};   // k_mean: read by bulk copies
   for (const void* p : a16)
     if (!aligned(p, 16)) return FQA_ERR_MISALIGNED;
-  const void* a4[] = {sq, sk, sv, sv_max};
+  const void* a4[] = {sq, sk, sv, sv_max, k_err};
   for (const void* p : a4)
     if (!aligned(p, 4)) return FQA_ERR_MISALIGNED;
   uint32_t* status = status_ptr(&st);
@@ -239,13 +240,31 @@ fqa_status fqa_quantize(const void* q, const void* k, const void* v, int B, int 
   uint8_t* v8b = static_cast<uint8_t*>(v8);
   void* args[] = {(void*)&qb, (void*)&kb, (void*)&vb, (void*)&q8b, (void*)&k8b, (void*)&v8b,
                   (void*)&sq, (void*)&sk, (void*)&sv, (void*)&sv_max, (void*)&k_mean,
-                  (void*)&partial, (void*)&ctr, (void*)&B, (void*)&H, (void*)&N, (void*)&status};
+                  (void*)&partial, (void*)&ctr, (void*)&B, (void*)&H, (void*)&N, (void*)&status,
+                  (void*)&k_err};
   // cooperative: every CTA is resident, so the grid barriers cannot wait on
   // a CTA that never starts
   if (cudaLaunchCooperativeKernel((const void*)quantize_fused_kernel, dim3(grid), dim3(kQuantThreads),
                                   args, kQuantSmem, s) != cudaSuccess)
     return FQA_ERR_CUDA;
   return launch_status();
+}
+
+fqa_status fqa_quantize(const void* q, const void* k, const void* v, int B, int H, int N, int d,
+                        void* q8, void* k8, void* v8, float* sq, float* sk, float* sv,
+                        float* sv_max, float* k_mean, void* workspace, size_t workspace_bytes,
+                        void* cuda_stream) {
+  return quantize_impl(q, k, v, B, H, N, d, q8, k8, v8, sq, sk, sv, sv_max, k_mean, nullptr, workspace,
+                       workspace_bytes, cuda_stream);
+}
+
+fqa_status fqa_quantize_keyerr(const void* q, const void* k, const void* v, int B, int H, int N, int d,
+                               void* q8, void* k8, void* v8, float* sq, float* sk, float* sv,
+                               float* sv_max, float* k_mean, float* k_err, void* workspace,
+                               size_t workspace_bytes, void* cuda_stream) {
+  if (k_err == nullptr) return FQA_ERR_INVALID_ARG;
+  return quantize_impl(q, k, v, B, H, N, d, q8, k8, v8, sq, sk, sv, sv_max, k_mean, k_err, workspace,
+                       workspace_bytes, cuda_stream);
 }
 
 static fqa_status check_attention_common(int B, int H, int N, int d, float softmax_scale,
@@ -299,6 +318,105 @@ fqa_status fqa_attention_bf16(const void* q, const void* k, const void* v, int B
   AttnParams prm{B, H, N, softmax_scale, nullptr, nullptr, nullptr, nullptr, out,
                  out_dtype == FQA_OUT_F32, status};
   return launch_attention_bf16(q, k, v, prm, static_cast<cudaStream_t>(cuda_stream));
+}
+
+// ---------------------------------------------------- error-corrected path
+
+// ceil(rho * N - 0.01): rho arrives in binary32, whose rounding moves rho * N
+// by at most 0.004 for N <= 65536, so a product meant to be an integer (0.05
+// of 1280 keys) stays that integer instead of rounding up.
+int fqa_corrected_keys(int N, float rho) {
+  if (N < 1 || !(rho >= 0.0f) || !(rho <= 1.0f)) return -1;
+  const double kc = std::ceil((double)rho * (double)N - 0.01);
+  return kc < 0.0 ? 0 : (kc > (double)N ? N : (int)kc);
+}
+
+static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+fqa_status fqa_select_keys(const float* k_err, int B, int H, int N, int kc, uint32_t* kmask, int* idx,
+                           void* cuda_stream) {
+  fqa_status st = check_shape(B, H, N, 128);
+  if (st != FQA_OK) return st;
+  if (k_err == nullptr || kmask == nullptr || kc < 1 || kc > N || (idx == nullptr)) return FQA_ERR_INVALID_ARG;
+  const void* a4[] = {k_err, kmask, idx};
+  for (const void* p : a4)
+    if (!aligned(p, 4)) return FQA_ERR_MISALIGNED;
+  if (!status_ptr(&st)) return st;
+  select_keys_kernel<<<B * H, kSelThreads, 0, static_cast<cudaStream_t>(cuda_stream)>>>(k_err, N, kc, kmask,
+                                                                                      idx);
+  return launch_status();
+}
+
+size_t fqa_attention_fp8_corrected_workspace_bytes(int B, int H, int N, int d, float rho) {
+  if (check_shape(B, H, N, d) != FQA_OK) return 0;
+  const int kc = fqa_corrected_keys(N, rho);
+  if (kc < 0) return 0;
+  const size_t rows = (size_t)B * H * N;
+  return align256((size_t)B * H * ((N + 31) / 32) * 4)      // key mask
+         + align256((size_t)B * H * (size_t)(kc > 0 ? kc : 1) * 4)   // corrected indices
+         + align256(rows * 8)                                // (m, l) per row
+         + align256(rows * 128 * 4);                         // FP8 part, FP32
+}
+
+fqa_status fqa_attention_fp8_corrected(const void* q, const void* k, const void* v, const void* q8,
+                                       const void* k8, const void* v8, const float* sq, const float* sk,
+                                       const float* sv, const float* sv_max, const float* k_mean,
+                                       const float* k_err, int B, int H, int N, int d, float softmax_scale,
+                                       float rho, void* out, fqa_out_dtype out_dtype, void* workspace,
+                                       size_t workspace_bytes, void* cuda_stream) {
+  fqa_status st = check_attention_common(B, H, N, d, softmax_scale, out, out_dtype);
+  if (st != FQA_OK) return st;
+  const int kc = fqa_corrected_keys(N, rho);
+  if (kc < 0) return FQA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, q8, k8, v8, sq, sk, sv, sv_max, k_mean, k_err, workspace};
+  for (const void* p : ptrs)
+    if (p == nullptr) return FQA_ERR_INVALID_ARG;
+  if (workspace_bytes < fqa_attention_fp8_corrected_workspace_bytes(B, H, N, d, rho))
+    return FQA_ERR_INVALID_ARG;
+  const void* a16[] = {q, k, v, q8, k8, v8, workspace};
+  for (const void* p : a16)
+    if (!aligned(p, 16)) return FQA_ERR_MISALIGNED;
+  const void* a4[] = {sq, sk, sv, sv_max, k_mean, k_err};
+  for (const void* p : a4)
+    if (!aligned(p, 4)) return FQA_ERR_MISALIGNED;
+  uint32_t* status = status_ptr(&st);
+  if (!status) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  if (kc == 0)   // nothing to correct: the plain FP8 path
+    return fqa_attention_fp8(q8, k8, v8, sq, sk, sv, sv_max, B, H, N, d, softmax_scale, out, out_dtype,
+                             cuda_stream);
+  // workspace: key mask | corrected indices | (m, l) | FP8 part (FP32)
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  uint32_t* kmask = reinterpret_cast<uint32_t*>(w);
+  w += align256((size_t)B * H * ((N + 31) / 32) * 4);
+  int* idx = reinterpret_cast<int*>(w);
+  w += align256((size_t)B * H * (size_t)kc * 4);
+  float2* stats = reinterpret_cast<float2*>(w);
+  w += align256((size_t)B * H * N * 8);
+  float* o1 = reinterpret_cast<float*>(w);
+  if ((st = fqa_select_keys(k_err, B, H, N, kc, kmask, idx, cuda_stream)) != FQA_OK) return st;
+  AttnParams prm{B, H, N, softmax_scale, sq, sk, sv, sv_max, o1, 1, status};
+  prm.q8 = static_cast<const uint8_t*>(q8);
+  prm.k8 = static_cast<const uint8_t*>(k8);
+  prm.kmask = kmask;
+  prm.row_stats = stats;
+  if ((st = launch_attention_fp8(q8, k8, v8, prm, s)) != FQA_OK) return st;
+  // exact part over the corrected keys, merged into the output
+  CUtensorMap tq;
+  if (!make_tmap(&tq, q, false, N, B * H)) return FQA_ERR_CUDA;
+  if (cudaFuncSetAttribute(correct_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           CorrTraits::kSmemBytes) != cudaSuccess)
+    return FQA_ERR_CUDA;
+  CorrParams cp{static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+                static_cast<const __nv_bfloat16*>(v), k_mean, idx, o1, stats, out,
+                out_dtype == FQA_OUT_F32, B, H, N, kc, softmax_scale, status};
+  const int sms = num_sms();
+  const int ntq = (N + 127) / 128;
+  int split = (sms + B * H - 1) / (B * H);       // about one wave of CTAs
+  if (split > ntq) split = ntq;
+  if (split < 1) split = 1;
+  correct_kernel<<<dim3(split, B * H), kCorrThreads, CorrTraits::kSmemBytes, s>>>(tq, cp);
+  return launch_status();
 }
 
 fqa_status fqa_e4m3_encode(const float* x, uint8_t* out, size_t n, void* cuda_stream) {

@@ -109,11 +109,28 @@ __device__ __forceinline__ void chunks_to_f32(const uint8_t* blk, int nvalid, fl
   }
 }
 
+// Residual squares of one chunk (8 consecutive channels): the sequential
+// binary32 sum of fl32(r^2), r = fl32(x - fl32(dec(code) * scale)), for the
+// four packed code pairs w[0..3] (element 2e in bits [0,8) of w[e]).
+__device__ __forceinline__ float residual_sq8(const float* x, const uint32_t (&w)[4], float scale) {
+  float acc = 0.0f;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 d = e4m3x2_to_f2(w[e]);
+    const float r0 = __fsub_rn(x[2 * e], __fmul_rn(d.x, scale));
+    const float r1 = __fsub_rn(x[2 * e + 1], __fmul_rn(d.y, scale));
+    acc = __fadd_rn(acc, __fmul_rn(r0, r0));
+    acc = __fadd_rn(acc, __fmul_rn(r1, r1));
+  }
+  return acc;
+}
+
 // Block absmax over the CTA (red: one float per warp for this slot), scale,
 // and the codes of this thread's chunks (8 bytes per chunk, chunk c at byte
-// 8c; chunks at or beyond nvalid are not stored).
+// 8c; chunks at or beyond nvalid are not stored).  rsq (optional): each
+// chunk's residual squares (residual_sq8).
 __device__ __forceinline__ float quantize_chunks(float (&x)[kVals], float* red, uint8_t* dst, int slot,
-                                                 int nvalid, uint64_t policy) {
+                                                 int nvalid, uint64_t policy, float* rsq = nullptr) {
   const int t = threadIdx.x;
   float m = 0.0f;
 #pragma unroll
@@ -139,6 +156,7 @@ __device__ __forceinline__ float quantize_chunks(float (&x)[kVals], float* red, 
         w[e] = e4m3x2(__fdiv_rn(x[8 * i + 2 * e], scale), __fdiv_rn(x[8 * i + 2 * e + 1], scale));
       if (t + kQuantThreads * i < nvalid)
         st_global_v2_hint(dst + 8 * (t + kQuantThreads * i), w[0] | (w[1] << 16), w[2] | (w[3] << 16), policy);
+      if (rsq) rsq[i] = residual_sq8(&x[8 * i], w, scale);
     }
     return scale;
   }
@@ -150,6 +168,10 @@ __device__ __forceinline__ float quantize_chunks(float (&x)[kVals], float* red, 
     uint32_t hi2 = e4m3x2(__fmul_rn(x[8 * i + 6], inv), __fmul_rn(x[8 * i + 7], inv));
     if (t + kQuantThreads * i < nvalid)
       st_global_v2_hint(dst + 8 * (t + kQuantThreads * i), lo | (hi << 16), lo2 | (hi2 << 16), policy);
+    if (rsq) {
+      const uint32_t w[4] = {lo, hi, lo2, hi2};
+      rsq[i] = residual_sq8(&x[8 * i], w, scale);
+    }
   }
   return scale;
 }
@@ -160,7 +182,7 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantMinCtas) quantize_fused_k
     uint8_t* __restrict__ v8, float* __restrict__ sq, float* __restrict__ sk,
     float* __restrict__ sv, float* __restrict__ sv_max, float* __restrict__ k_mean,
     float* __restrict__ partial, unsigned int* __restrict__ ctr, int B, int H, int N,
-    uint32_t* status) {
+    uint32_t* status, float* __restrict__ k_err) {
   extern __shared__ uint8_t qsmem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(qsmem_raw) + 127) & ~uintptr_t(127));
   __shared__ uint64_t full[kMaxSlots];
@@ -355,8 +377,29 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantMinCtas) quantize_fused_k
             for (int e = 0; e < 8; ++e) x[8 * i4 + e] = __fsub_rn(x[8 * i4 + e], mr[e]);
           }
         }
-        const float s_k = quantize_chunks(x, red, k8 + unit_off(u), 0, nvalid, pol_first);
+        if (k_err == nullptr) {
+          const float s_k = quantize_chunks(x, red, k8 + unit_off(u), 0, nvalid, pol_first);
+          if (t == 0) sk[u] = s_k;
+          return;
+        }
+        // with the per-key quantization error: chunk i of this thread is
+        // channels 8 (t % 16) .. +8 of token t / 16 + 16 i of the unit; the 16
+        // lanes of a token combine their chunk sums pairwise in the pinned
+        // order g_l + g_l^8, then ^4, ^2, ^1 (identical in every lane)
+        float rsq[kChunks];
+        const float s_k = quantize_chunks(x, red, k8 + unit_off(u), 0, nvalid, pol_first, rsq);
         if (t == 0) sk[u] = s_k;
+        const size_t tok0 = unit_off(u) / kHeadDim;
+#pragma unroll
+        for (int i = 0; i < kChunks; ++i) {
+          float e = rsq[i];
+          e = __fadd_rn(e, __shfl_xor_sync(0xffffffffu, e, 8));
+          e = __fadd_rn(e, __shfl_xor_sync(0xffffffffu, e, 4));
+          e = __fadd_rn(e, __shfl_xor_sync(0xffffffffu, e, 2));
+          e = __fadd_rn(e, __shfl_xor_sync(0xffffffffu, e, 1));
+          const int c = t + kQuantThreads * i;
+          if ((t & 15) == 0 && c < nvalid) k_err[tok0 + c / 16] = e;
+        }
       });
 }
 

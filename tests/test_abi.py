@@ -113,3 +113,18 @@ def test_attention_validation(L):
     L.fqa_debug_wait_timeout.argtypes = [ctypes.c_uint32, P]
     assert L.fqa_debug_wait_timeout(0, None) == 1
     assert L.fqa_debug_wait_timeout(3000000, None) == 1
+
+
+def test_corrected_key_count_matches_the_oracle(L):
+    """The count of corrected keys per head is a host computation on the
+    binary32 rho the ABI takes; it must agree with the oracle's reading."""
+    import oracle
+    import quantized_fp8_attention_b200 as fqa
+    for N in (1, 7, 100, 200, 1000, 1280, 4429, 4608, 8704, 16896, 65536):
+        for rho in (0.0, 0.001, 0.005, 0.01, 0.02, 0.05, 0.1, 0.25, 0.5, 1.0):
+            assert fqa.fqa_corrected_keys(N, rho) == oracle.n_corrected(N, rho), (N, rho)
+    assert fqa.fqa_corrected_keys(0, 0.1) == -1
+    assert fqa.fqa_corrected_keys(100, 1.5) == -1
+    assert fqa.fqa_corrected_keys(100, float("nan")) == -1
+    assert fqa.fqa_attention_fp8_corrected_workspace_bytes(1, 24, 8704, 0.005) > 24 * 8704 * 512
+    assert fqa.fqa_attention_fp8_corrected_workspace_bytes(1, 24, 8704, 2.0) == 0

@@ -99,9 +99,11 @@ def test_select_keys_brute_force_with_ties():
 def test_n_corrected_rounds_up():
     assert oracle.n_corrected(8704, 0.005) == 44
     assert oracle.n_corrected(1280, 0.005) == 7
+    assert oracle.n_corrected(1280, 0.05) == 64      # fl32(0.05) * 1280 = 64.000001
     assert oracle.n_corrected(100, 0.0) == 0
     assert oracle.n_corrected(100, 1.0) == 100
     assert oracle.n_corrected(200, 0.005) == 1
+    assert oracle.n_corrected(65536, 0.005) == 328
 
 
 # ----------------------------------------------------- corrected attention
