@@ -216,6 +216,13 @@ def run_sweep(args):
         ms_a = timed(lambda: fqa.attention_fp8(qz, scale, fqa.FQA_OUT_BF16, out=out), reps(1200))
         ms_b = timed(lambda: fqa.attention_bf16(q, k, v, scale, fqa.FQA_OUT_BF16, out=out), reps(850))
         ms_q = timed(lambda: fqa.quantize(q, k, v, out=qz, workspace=ws), 200, pre=lambda: flush.fill_(1))
+        # error-corrected attention (rho = 0.005) on the same codes: selection,
+        # masked FP8 attention, exact part and merge
+        k_err = torch.empty(w.B, w.H, w.N, dtype=torch.float32, device=dev)
+        fqa.quantize_keyerr(q, k, v, out=qz, k_err=k_err, workspace=ws)
+        cws = fqa.alloc_corrected_workspace(w.B, w.H, w.N, 0.005, dev)
+        ms_c = timed(lambda: fqa.attention_fp8_corrected(q, k, v, qz, k_err, scale, 0.005, fqa.FQA_OUT_BF16,
+                                                         out=out, workspace=cws), reps(1000))
         st, flags = fqa.fqa_debug_status()
         if st != fqa.FQA_OK:
             raise RuntimeError(f"device status {flags:#x} on {w.name}")
@@ -225,18 +232,20 @@ def run_sweep(args):
             "sweep": True, "workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
             "attention_fp8": {"ms": ms_a, "tflops": w.flops / ms_a / 1e9,
                               "frac_of_fp8_peak": w.flops / ms_a / 1e9 / fp8_peak},
+            "attention_fp8_corrected": {"ms": ms_c, "rho": 0.005, "keys_per_head": fqa.fqa_corrected_keys(w.N, 0.005),
+                                        "time_vs_fp8": ms_c / ms_a, "time_vs_bf16": ms_c / ms_b},
             "attention_bf16": {"ms": ms_b, "tflops": w.flops / ms_b / 1e9,
                                "frac_of_bf16_peak": w.flops / ms_b / 1e9 / pk["bf16_tflops"]},
             "quantizer": {"ms": ms_q, "gbs": qbytes / ms_q / 1e6, "frac_of_hbm": qbytes / ms_q / 1e6 / pk["hbm_gbs"],
                           "l2": "flushed before every launch"},
             "peaks": pk_kind}), flush=True)
-        del q, k, v, qz, ws, out
+        del q, k, v, qz, ws, out, k_err, cws
         torch.cuda.empty_cache()
 
 
 def step_line(w, world: int, K: int, warmup: int, ms_per_step: float, attn_ms: float, quant_ms: float,
               bf16_ms: float, e2e_ms: float, h2d: int, d2h: int, clocks: dict, probe, cpu, traffic,
-              pk: dict, pk_kind: str) -> dict:
+              pk: dict, pk_kind: str, corrected=None, accuracy=None) -> dict:
     """The benchmark's JSON line for workload w from the measured times (ms).
     value and e2e are whole-job throughput (every rank runs its own batch);
     roofline is for the FP8 attention kernel against 2 x the measured BF16
@@ -277,7 +286,39 @@ def step_line(w, world: int, K: int, warmup: int, ms_per_step: float, attn_ms: f
         "clocks": clocks,
         "fp8_gemm_probe": probe,
         "cpu_baseline": cpu,
+        "corrected": corrected,
+        "accuracy": accuracy,
     }
+
+
+# ----------------------------------------------------------------- accuracy
+
+def accuracy_sample(w, g, q, k, v, scale, rho, qz, k_err, out, cws):
+    """Cosine against exact FP64 attention (the CPU oracle) on 2 heads x 384
+    rows of the workload, for the plain FP8 path and the corrected path, with
+    the 0.995 target flagged.  Runs outside the timed region."""
+    import torch
+
+    import oracle
+    import quantized_fp8_attention_b200 as fqa
+    heads = [(0, 0), (0, w.H - 1)]
+    rows = list(range(0, 128)) + list(range(w.N // 2, w.N // 2 + 128)) + list(range(w.N - 128, w.N))
+    ex = oracle.attention_exact(g["q"], g["k"], g["v"], scale, heads=heads, rows=rows)
+
+    def cos(t):
+        a = t.float().cpu().numpy()
+        got = np.stack([a[b, h][rows] for (b, h) in heads]).astype(np.float64)
+        return float((got * ex).sum() / np.sqrt((got * got).sum() * (ex * ex).sum()))
+
+    fqa.quantize(q, k, v, out=qz)
+    plain = cos(fqa.attention_fp8(qz, scale, fqa.FQA_OUT_F32))
+    fqa.quantize_keyerr(q, k, v, out=qz, k_err=k_err)
+    corr = cos(fqa.attention_fp8_corrected(q, k, v, qz, k_err, scale, rho, fqa.FQA_OUT_F32, workspace=cws))
+    sample = f"heads {heads}, rows [0,128) u [N/2, N/2+128) u [N-128, N), all keys"
+    accuracy = {"cos_vs_exact_fp64": plain, "target": 0.995, "meets_target": plain >= 0.995, "sample": sample}
+    corrected = {"rho": rho, "keys_per_head": fqa.fqa_corrected_keys(w.N, rho), "cos_vs_exact_fp64": corr,
+                 "meets_target": corr >= 0.995}
+    return accuracy, corrected
 
 
 # ------------------------------------------------------------ CPU baseline
@@ -469,13 +510,40 @@ def run_fqa(args, rank: int, world: int):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / Ke, dev, world)
 
+    # error-corrected FP8 attention at the pages' rho, same inputs: the quantizer
+    # with the key error, selection, masked FP8 attention, exact part + merge
+    rho = 0.005
+    k_err = torch.empty(B, H, N, dtype=torch.float32, device=dev)
+    cws = fqa.alloc_corrected_workspace(B, H, N, rho, dev)
+
+    def corrected_step():
+        fqa.quantize_keyerr(q, k, v, out=qz, k_err=k_err, workspace=ws)
+        fqa.attention_fp8_corrected(q, k, v, qz, k_err, scale, rho, fqa.FQA_OUT_BF16, out=out, workspace=cws)
+
+    for _ in range(3):
+        corrected_step()
+    Kc = max(1, K // 2)
+    e0.record(stream)
+    for _ in range(Kc):
+        corrected_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    corr_ms = e0.elapsed_time(e1) / Kc
+    st, flags = fqa.fqa_debug_status()
+    if st != fqa.FQA_OK:
+        raise RuntimeError(f"device status {flags:#x} after the corrected steps")
+
     if rank != 0:
         return
     pk, pk_kind = peaks()
     probe = fp8_gemm_probe(dev)
+    accuracy, corrected = accuracy_sample(w, g, q, k, v, scale, rho, qz, k_err, out, cws)
+    corrected.update({"ms_per_step": corr_ms, "step": "fqa_quantize_keyerr + fqa_attention_fp8_corrected",
+                      "tflops": flops / (corr_ms * 1e-3) / 1e12,
+                      "time_vs_fp8_step": corr_ms / ms_per_step, "time_vs_bf16_attention": corr_ms / bf16_ms})
     cpu = None if args.no_cpu_baseline else cpu_baseline(w, g)
     line = step_line(w, world, K, args.warmup, ms_per_step, attn_ms, quant_ms, bf16_ms, e2e_ms, h2d, d2h,
-                     clk.summary(), probe, cpu, traffic_per_launch(), pk, pk_kind)
+                     clk.summary(), probe, cpu, traffic_per_launch(), pk, pk_kind, corrected, accuracy)
     print(json.dumps(line), flush=True)
 
 
