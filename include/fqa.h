@@ -229,6 +229,36 @@ FQA_API fqa_status fqa_attention_bf16(const void* q, const void* k, const void* 
                               void* cuda_stream);
 
 /*
+ * Sequence-parallel (Ulysses) layouts.  [KLEIN] section "결과" and "고를 때
+ * 기준": multi-GPU runs split the CFG pair across GPU groups and shard each
+ * sequence over the GPUs of a group (Ulysses, degree 4 or 8), with an
+ * all-to-all that turns a sequence shard into a head shard before attention
+ * and back after it.  With P ranks in a group, rank r holding tokens
+ * [r Nl, (r+1) Nl) of all H = P * Hl heads, the all-to-all delivers to rank
+ * r its Hl heads for every token as P chunks: the layout
+ *   [B, P, Hl, Nl, d]   (chunk p: tokens [p Nl, (p+1) Nl) of the Hl heads).
+ * The two calls below read and write that layout directly, so no separate
+ * pack or unpack pass runs around the collectives.  Nl must be a multiple of
+ * 64 (no quantization block straddles two chunks); N = P * Nl.
+ */
+
+/* fqa_quantize() on inputs q, k, v in the layout [B, P, Hl, Nl, d]; every
+ * output in the usual layouts for B, Hl heads and N = P * Nl tokens.  Codes
+ * and scales are bit-identical to fqa_quantize() on the same tokens. */
+FQA_API fqa_status fqa_quantize_a2a(const void* q, const void* k, const void* v, int B, int Hl, int P, int Nl,
+                                    int d, void* q8, void* k8, void* v8, float* sq, float* sk, float* sv,
+                                    float* sv_max, float* k_mean, void* workspace, size_t workspace_bytes,
+                                    void* cuda_stream);
+
+/* fqa_attention_fp8() for B, Hl heads and N = P * Nl tokens, with out written
+ * in the layout [B, P, Hl, Nl, d] (ready for the return all-to-all);
+ * bit-identical values to fqa_attention_fp8(). */
+FQA_API fqa_status fqa_attention_fp8_a2a(const void* q8, const void* k8, const void* v8, const float* sq,
+                                         const float* sk, const float* sv, const float* sv_max, int B, int Hl,
+                                         int P, int Nl, int d, float softmax_scale, void* out,
+                                         fqa_out_dtype out_dtype, void* cuda_stream);
+
+/*
  * Error-corrected FP8 attention: FP8 attention that corrects only the tokens
  * with large error.  [KLEIN] section "왜 이런 차이가 나나": VC-Attention FP8
  * (rho = 0.005) is one of the B200 FP8 attention backends measured there; the

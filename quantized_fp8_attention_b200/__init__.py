@@ -54,6 +54,10 @@ def _load():
     L.fqa_e4m3_encode.argtypes = [P, P, ctypes.c_size_t, P]
     L.fqa_debug_status.restype = I
     L.fqa_debug_status.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
+    L.fqa_quantize_a2a.restype = I
+    L.fqa_quantize_a2a.argtypes = [P, P, P, I, I, I, I, I, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+    L.fqa_attention_fp8_a2a.restype = I
+    L.fqa_attention_fp8_a2a.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, ctypes.c_float, P, I, P]
     L.fqa_quantize_keyerr.restype = I
     L.fqa_quantize_keyerr.argtypes = [P, P, P, I, I, I, I, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
     L.fqa_corrected_keys.restype = I
@@ -143,6 +147,23 @@ def fqa_attention_bf16(q, k, v, softmax_scale, out, out_dtype, stream=None) -> i
     B, H, N, d = q.shape
     return _load().fqa_attention_bf16(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, float(softmax_scale),
                                    _ptr(out), int(out_dtype), _stream(stream))
+
+
+def fqa_quantize_a2a(q, k, v, q8, k8, v8, sq, sk, sv, sv_max, k_mean, workspace, stream=None) -> int:
+    """fqa_quantize on inputs in the sequence all-to-all layout [B, P, Hl, Nl, d]."""
+    B, P, Hl, Nl, d = q.shape
+    return _load().fqa_quantize_a2a(_ptr(q), _ptr(k), _ptr(v), B, Hl, P, Nl, d, _ptr(q8), _ptr(k8), _ptr(v8),
+                                 _ptr(sq), _ptr(sk), _ptr(sv), _ptr(sv_max), _ptr(k_mean), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream(stream))
+
+
+def fqa_attention_fp8_a2a(q8, k8, v8, sq, sk, sv, sv_max, P: int, softmax_scale, out, out_dtype,
+                          stream=None) -> int:
+    """fqa_attention_fp8 writing out in the layout [B, P, Hl, N / P, d]."""
+    B, Hl, N, d = q8.shape
+    return _load().fqa_attention_fp8_a2a(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(sq), _ptr(sk), _ptr(sv),
+                                      _ptr(sv_max), B, Hl, int(P), N // int(P), d, float(softmax_scale),
+                                      _ptr(out), int(out_dtype), _stream(stream))
 
 
 def fqa_quantize_keyerr(q, k, v, q8, k8, v8, sq, sk, sv, sv_max, k_mean, k_err, workspace,
@@ -320,6 +341,43 @@ def quantize_keyerr(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: Opti
     _require(workspace, workspace.dtype, "workspace")
     _check(fqa_quantize_keyerr(q, k, v, *out, k_err, workspace, stream=stream), "fqa_quantize_keyerr")
     return out, k_err
+
+
+def quantize_a2a(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: Optional[Quantized] = None,
+                 workspace: Optional[torch.Tensor] = None, stream=None) -> Quantized:
+    """Q, K, V in the sequence all-to-all layout [B, P, Hl, Nl, 128] (BF16,
+    CUDA, contiguous; Nl a multiple of 64) -> Quantized for B, Hl heads and
+    N = P * Nl tokens in the usual layouts."""
+    if not isinstance(q, torch.Tensor) or q.dim() != 5:
+        raise ValueError("q: expected a [B, P, Hl, Nl, 128] tensor")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _require(t, torch.bfloat16, name, q.shape)
+    B, P, Hl, Nl, _ = q.shape
+    N = P * Nl
+    if out is None:
+        out = alloc_quantized(B, Hl, N, q.device)
+    _require_quantized(out, B, Hl, N)
+    if workspace is None:
+        workspace = alloc_workspace(B, Hl, N, q.device)
+    _require(workspace, workspace.dtype, "workspace")
+    _check(fqa_quantize_a2a(q, k, v, *out, workspace, stream=stream), "fqa_quantize_a2a")
+    return out
+
+
+def attention_fp8_a2a(qz: Quantized, P: int, softmax_scale: float, out_dtype: int = FQA_OUT_BF16,
+                      out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """fqa_attention_fp8 with the output in the layout [B, P, Hl, N / P, 128]."""
+    B, Hl, N, d = qz.q8.shape
+    _require_quantized(qz, B, Hl, N)
+    if N % P:
+        raise ValueError(f"N = {N} is not a multiple of P = {P}")
+    dt = torch.float32 if out_dtype == FQA_OUT_F32 else torch.bfloat16
+    if out is None:
+        out = torch.empty(B, P, Hl, N // P, d, dtype=dt, device=qz.q8.device)
+    _require(out, dt, "out", (B, P, Hl, N // P, d))
+    _check(fqa_attention_fp8_a2a(*qz[:7], P, softmax_scale, out, out_dtype, stream=stream),
+           "fqa_attention_fp8_a2a")
+    return out
 
 
 def alloc_corrected_workspace(B: int, H: int, N: int, rho: float, device) -> torch.Tensor:

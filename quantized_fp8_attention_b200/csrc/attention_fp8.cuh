@@ -548,6 +548,13 @@ __global__ void __launch_bounds__(kF8Threads, 1)
         if (p.row_stats != nullptr && hf == 0 && store) p.row_stats[orow] = make_float2(m, l_row);
       }
 #pragma unroll 1
+      // the output row: [B,H,N,128], or with out_P > 1 the sequence all-to-all
+      // layout [B, out_P, H, N / out_P, 128] (chunk c: tokens [c N/out_P, ...))
+      size_t orow_out = orow;
+      if (p.out_P > 1) {
+        const int nl = N / p.out_P, cq = qrow / nl;
+        orow_out = (((size_t)w.b * p.out_P + cq) * p.H + w.h) * nl + (qrow - cq * nl);
+      }
       for (int c = 0; c < 2; ++c) {
         uint32_t o[32];
         const int col = 64 * hf + 32 * c;
@@ -555,14 +562,14 @@ __global__ void __launch_bounds__(kF8Threads, 1)
         tmem_wait_ld();
         if (!store) continue;
         if (p.out_f32) {
-          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow * 128 + col);
+          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow_out * 128 + col);
 #pragma unroll
           for (int e = 0; e < 8; ++e)
             dst[e] = make_float4(__uint_as_float(o[4 * e]) * fin, __uint_as_float(o[4 * e + 1]) * fin,
                                  __uint_as_float(o[4 * e + 2]) * fin,
                                  __uint_as_float(o[4 * e + 3]) * fin);
         } else {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + orow * 128 + col);
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + orow_out * 128 + col);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             uint32_t w4[4];

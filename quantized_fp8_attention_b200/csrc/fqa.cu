@@ -200,7 +200,7 @@ size_t fqa_quantize_workspace_bytes(int B, int H, int N, int d) {
 static fqa_status quantize_impl(const void* q, const void* k, const void* v, int B, int H, int N, int d,
                                 void* q8, void* k8, void* v8, float* sq, float* sk, float* sv,
                                 float* sv_max, float* k_mean, float* k_err, void* workspace,
-                                size_t workspace_bytes, void* cuda_stream) {
+                                size_t workspace_bytes, void* cuda_stream, int in_P = 1) {
   fqa_status st = check_shape(B, H, N, d);
   if (st != FQA_OK) return st;
   const void* ptrs[] = {q, k, v, q8, k8, v8, sq, sk, sv, sv_max, k_mean, workspace};
@@ -241,7 +241,7 @@ static fqa_status quantize_impl(const void* q, const void* k, const void* v, int
   void* args[] = {(void*)&qb, (void*)&kb, (void*)&vb, (void*)&q8b, (void*)&k8b, (void*)&v8b,
                   (void*)&sq, (void*)&sk, (void*)&sv, (void*)&sv_max, (void*)&k_mean,
                   (void*)&partial, (void*)&ctr, (void*)&B, (void*)&H, (void*)&N, (void*)&status,
-                  (void*)&k_err};
+                  (void*)&k_err, (void*)&in_P};
   // cooperative: every CTA is resident, so the grid barriers cannot wait on
   // a CTA that never starts
   if (cudaLaunchCooperativeKernel((const void*)quantize_fused_kernel, dim3(grid), dim3(kQuantThreads),
@@ -318,6 +318,53 @@ fqa_status fqa_attention_bf16(const void* q, const void* k, const void* v, int B
   AttnParams prm{B, H, N, softmax_scale, nullptr, nullptr, nullptr, nullptr, out,
                  out_dtype == FQA_OUT_F32, status};
   return launch_attention_bf16(q, k, v, prm, static_cast<cudaStream_t>(cuda_stream));
+}
+
+// ------------------------------------------- sequence all-to-all layouts
+
+// Shapes of the all-to-all calls: B, Hl heads, P chunks of Nl tokens
+// (N = P * Nl), Nl a multiple of 64 so that no quantization block straddles
+// two chunks.
+static fqa_status check_a2a(int B, int Hl, int P, int Nl, int d) {
+  if (P < 1 || Nl < 1) return FQA_ERR_INVALID_ARG;
+  if (Nl % kQBlock != 0) return FQA_ERR_UNSUPPORTED;
+  if ((int64_t)P * Nl > 65536) return FQA_ERR_UNSUPPORTED;
+  return check_shape(B, Hl, P * Nl, d);
+}
+
+fqa_status fqa_quantize_a2a(const void* q, const void* k, const void* v, int B, int Hl, int P, int Nl, int d,
+                            void* q8, void* k8, void* v8, float* sq, float* sk, float* sv, float* sv_max,
+                            float* k_mean, void* workspace, size_t workspace_bytes, void* cuda_stream) {
+  fqa_status st = check_a2a(B, Hl, P, Nl, d);
+  if (st != FQA_OK) return st;
+  return quantize_impl(q, k, v, B, Hl, P * Nl, d, q8, k8, v8, sq, sk, sv, sv_max, k_mean, nullptr, workspace,
+                       workspace_bytes, cuda_stream, P);
+}
+
+fqa_status fqa_attention_fp8_a2a(const void* q8, const void* k8, const void* v8, const float* sq,
+                                 const float* sk, const float* sv, const float* sv_max, int B, int Hl, int P,
+                                 int Nl, int d, float softmax_scale, void* out, fqa_out_dtype out_dtype,
+                                 void* cuda_stream) {
+  fqa_status st = check_a2a(B, Hl, P, Nl, d);
+  if (st != FQA_OK) return st;
+  const int N = P * Nl;
+  if ((st = check_attention_common(B, Hl, N, d, softmax_scale, out, out_dtype)) != FQA_OK) return st;
+  const void* ptrs[] = {q8, k8, v8, sq, sk, sv, sv_max};
+  for (const void* p : ptrs)
+    if (p == nullptr) return FQA_ERR_INVALID_ARG;
+  const void* a16[] = {q8, k8, v8};
+  for (const void* p : a16)
+    if (!aligned(p, 16)) return FQA_ERR_MISALIGNED;
+  const void* a4[] = {sq, sk, sv, sv_max};
+  for (const void* p : a4)
+    if (!aligned(p, 4)) return FQA_ERR_MISALIGNED;
+  uint32_t* status = status_ptr(&st);
+  if (!status) return st;
+  AttnParams prm{B, Hl, N, softmax_scale, sq, sk, sv, sv_max, out, out_dtype == FQA_OUT_F32, status};
+  prm.q8 = static_cast<const uint8_t*>(q8);
+  prm.k8 = static_cast<const uint8_t*>(k8);
+  prm.out_P = P;
+  return launch_attention_fp8(q8, k8, v8, prm, static_cast<cudaStream_t>(cuda_stream));
 }
 
 // ---------------------------------------------------- error-corrected path

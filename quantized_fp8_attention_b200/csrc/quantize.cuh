@@ -182,7 +182,7 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantMinCtas) quantize_fused_k
     uint8_t* __restrict__ v8, float* __restrict__ sq, float* __restrict__ sk,
     float* __restrict__ sv, float* __restrict__ sv_max, float* __restrict__ k_mean,
     float* __restrict__ partial, unsigned int* __restrict__ ctr, int B, int H, int N,
-    uint32_t* status, float* __restrict__ k_err) {
+    uint32_t* status, float* __restrict__ k_err, int in_P) {
   extern __shared__ uint8_t qsmem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(qsmem_raw) + 127) & ~uintptr_t(127));
   __shared__ uint64_t full[kMaxSlots];
@@ -250,10 +250,23 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantMinCtas) quantize_fused_k
       return reverse ? nunits - 1 - (int)i : (int)i;
     };
   };
-  // element offset of unit u in a [B,H,N,128] tensor, and its token count
+  // element offset of unit u in a [B,H,N,128] tensor (the codes, and the
+  // inputs when in_P == 1), and its token count
   auto unit_off = [&](int u) {
     const int hd = u / nblk;
     return ((size_t)hd * N + (size_t)(u - hd * nblk) * kQBlock) * kHeadDim;
+  };
+  // element offset of unit u in the inputs: with in_P > 1 they are in the
+  // sequence all-to-all layout [B, in_P, H, N / in_P, 128] (chunk p holds
+  // tokens [p N/in_P, (p+1) N/in_P) of every head; N / in_P is a multiple of
+  // 64, so no block straddles two chunks)
+  const int nl = N / in_P;
+  auto unit_in = [&](int u) -> size_t {
+    if (in_P == 1) return unit_off(u);
+    const int hd = u / nblk;
+    const int n0 = (u - hd * nblk) * kQBlock, c = n0 / nl;
+    const int b = hd / H, h = hd - b * H;
+    return ((((size_t)b * in_P + c) * H + h) * nl + (n0 - c * nl)) * kHeadDim;
   };
   auto unit_rows = [&](int u) { return min(kQBlock, N - (u % nblk) * kQBlock); };
 
@@ -262,8 +275,8 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantMinCtas) quantize_fused_k
       [&](int u, uint8_t* dst, uint64_t* bar) {
         const uint32_t bytes = (uint32_t)unit_rows(u) * kHeadDim * 2;
         mbar_arrive_expect_tx(bar, 2 * bytes);
-        bulk_load(dst, q + unit_off(u), bytes, bar, pol_first);
-        bulk_load(dst + kBlockBytes, v + unit_off(u), bytes, bar, pol_first);
+        bulk_load(dst, q + unit_in(u), bytes, bar, pol_first);
+        bulk_load(dst + kBlockBytes, v + unit_in(u), bytes, bar, pol_first);
       },
       [&](int u, const uint8_t* blk) {
         const size_t off = unit_off(u);
@@ -285,7 +298,7 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantMinCtas) quantize_fused_k
         [&](int u, uint8_t* dst, uint64_t* bar) {
           const uint32_t bytes = (uint32_t)unit_rows(u) * kHeadDim * 2;
           mbar_arrive_expect_tx(bar, bytes);
-          bulk_load(dst, k + unit_off(u), bytes, bar, pol_last);
+          bulk_load(dst, k + unit_in(u), bytes, bar, pol_last);
         },
         [&](int u, const uint8_t* blk) {
           if (t < kHeadDim) {
@@ -357,7 +370,7 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantMinCtas) quantize_fused_k
       [&](int u, uint8_t* dst, uint64_t* bar) {
         const uint32_t bytes = (uint32_t)unit_rows(u) * kHeadDim * 2;
         mbar_arrive_expect_tx(bar, bytes + kHeadDim * 4);
-        bulk_load(dst, k + unit_off(u), bytes, bar, pol_first);
+        bulk_load(dst, k + unit_in(u), bytes, bar, pol_first);
         bulk_load(dst + kBlockBytes, k_mean + (size_t)(u / nblk) * kHeadDim, kHeadDim * 4, bar, pol_first);
       },
       [&](int u, const uint8_t* blk) {
