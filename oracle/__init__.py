@@ -75,6 +75,13 @@ def lib():
                                                   ctypes.c_float, i, P, i, P, i, P, P]
         L.orc_attention_fp8_part.argtypes = [P, P, P, P, P, P, P, P, i, i, i, i, ctypes.c_float, P, i, P, i,
                                              P, P, P]
+        L.orc_e2m1_decode.restype = ctypes.c_double
+        L.orc_e2m1_decode.argtypes = [ctypes.c_uint8]
+        L.orc_e2m1_encode.restype = ctypes.c_uint8
+        L.orc_e2m1_encode.argtypes = [ctypes.c_double]
+        L.orc_quantize_nvfp4_qk.argtypes = [P, P, P, i, i, i, i, P, P, P, P, P, P]
+        L.orc_attention_nvfp4.argtypes = [P, P, P, P, P, P, P, P, P, i, i, i, i, ctypes.c_float, P, i, P, i,
+                                          P, P, P]
         L.orc_e4m3_encode_f32_array.argtypes = [P, ctypes.c_size_t, P]
         L.orc_bf16_round_array.argtypes = [P, ctypes.c_size_t, P]
         L.orc_num_threads.restype = i
@@ -202,6 +209,49 @@ def attention_core(qc, kc, vc, sq, sk, sv, sv_max, scale, bc=128, quantize_p=Tru
                              N, d, float(scale), bc, int(bool(quantize_p)), _p(ra), len(ra),
                              _p(out), None if amb is None else _p(amb),
                              None if namb is None else _p(namb))
+    return (out, amb, namb) if with_ambiguity else out
+
+
+# ------------------------------------------------------------ NVFP4 Q.K
+
+def e2m1_decode(codes) -> np.ndarray:
+    codes = np.asarray(codes, dtype=np.uint8)
+    table = np.array([lib().orc_e2m1_decode(i) for i in range(16)], dtype=np.float64)
+    return table[codes & 15]
+
+
+def e2m1_encode_f64(x: float) -> int:
+    return int(lib().orc_e2m1_encode(float(x)))
+
+
+def quantize_nvfp4(q: np.ndarray, k: np.ndarray, v: np.ndarray) -> dict:
+    """The FP8 quantizer's outputs (V codes, scales, k_mean) plus Q and
+    smoothed K in NVFP4: q4/k4 [B,H,N,64] packed E2M1 (element 2i in the low
+    nibble), sfq/sfk [B,H,N,8] E4M3 group scales, sq1/sk1 [B,H,ceil(N/64)]."""
+    r = quantize(q, k, v)
+    B, H, N, d = q.shape
+    nb = (N + 63) // 64
+    q = np.ascontiguousarray(q, dtype=np.uint16)
+    k = np.ascontiguousarray(k, dtype=np.uint16)
+    r.update(q4=np.empty((B, H, N, d // 2), np.uint8), k4=np.empty((B, H, N, d // 2), np.uint8),
+             sfq=np.empty((B, H, N, d // 16), np.uint8), sfk=np.empty((B, H, N, d // 16), np.uint8),
+             sq1=np.empty((B, H, nb), np.float32), sk1=np.empty((B, H, nb), np.float32))
+    lib().orc_quantize_nvfp4_qk(_p(q), _p(k), _p(r["k_mean"]), B, H, N, d, _p(r["q4"]), _p(r["k4"]),
+                                _p(r["sfq"]), _p(r["sfk"]), _p(r["sq1"]), _p(r["sk1"]))
+    return r
+
+
+def attention_nvfp4(qz: dict, softmax_scale: float, heads=None, rows=None, with_ambiguity: bool = False):
+    """NVFP4 Q.K, FP8 P.V attention on quantize_nvfp4() outputs -> [n_heads, n_rows, d]."""
+    B, H, N, d = qz["v8"].shape
+    ha, ra = _heads_rows(B, H, N, heads, rows)
+    out = np.empty((len(ha), len(ra), d), dtype=np.float64)
+    amb = np.empty_like(out) if with_ambiguity else None
+    namb = np.empty((len(ha), len(ra)), dtype=np.int32) if with_ambiguity else None
+    lib().orc_attention_nvfp4(_p(qz["q4"]), _p(qz["k4"]), _p(qz["sfq"]), _p(qz["sfk"]), _p(qz["sq1"]),
+                              _p(qz["sk1"]), _p(qz["v8"]), _p(qz["sv"]), _p(qz["sv_max"]), B, H, N, d,
+                              float(np.float32(softmax_scale)), _p(ha), len(ha), _p(ra), len(ra), _p(out),
+                              None if amb is None else _p(amb), None if namb is None else _p(namb))
     return (out, amb, namb) if with_ambiguity else out
 
 

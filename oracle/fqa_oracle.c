@@ -397,6 +397,156 @@ void orc_attention_fp8(const uint8_t *q8, const uint8_t *k8, const uint8_t *v8,
     free(qc); free(kc); free(vc);
 }
 
+/* ------------------------------------------------- NVFP4 Q and K (FP4) */
+/* The FP4 scheme: "NVIDIA RTX AI optimiert FLUX.1 fuer Bilddaten mit
+ * niedriger Genauigkeit", SDPA quantization paragraph (the FP8 and FP4
+ * schemes differ only in the precision of the Q, K, V projections; attention
+ * itself stays in FP8).  The pages name no FP4 format; the reading is NVFP4
+ * for the Q and K operands of Q K^T -- E2M1 elements with one unsigned E4M3
+ * scale per 16 consecutive channels -- on top of the FP8 path's per-(b, h,
+ * 64-token block) FP32 scale; V, P and P.V stay FP8. */
+
+/* E2M1 value of a 4-bit code: sign in bit 3, exponent bits [1,3) (bias 1),
+ * mantissa bit 0; subnormal 0.5 for exponent 0.  Values 0, 0.5, 1, 1.5, 2, 3,
+ * 4, 6. */
+double orc_e2m1_decode(uint8_t code)
+{
+    int sign = (code >> 3) & 1, e = (code >> 1) & 3, m = code & 1;
+    double v = e == 0 ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    return sign ? -v : v;
+}
+
+/* E2M1, round to nearest (ties to the even code), saturating to +-6; the
+ * sign of zero is kept.  x must not be NaN.  Nearest-even over the table. */
+uint8_t orc_e2m1_encode(double x)
+{
+    uint8_t sign = signbit(x) ? 0x8 : 0x0;
+    double a = fabs(x);
+    if (a >= 6.0)
+        return sign | 7;
+    int best = 0;
+    double bd = INFINITY;
+    for (int c = 0; c < 8; c++) {
+        double dlt = fabs(orc_e2m1_decode((uint8_t)c) - a);
+        if (dlt < bd || (dlt == bd && (c & 1) == 0 && (best & 1) == 1)) {
+            bd = dlt;
+            best = c;
+        }
+    }
+    return sign | (uint8_t)best;
+}
+
+/* One block (n_tok tokens x d channels, x binary32, K already smoothed) in
+ * NVFP4 [reading, pinned binary32 order]:
+ *   s1  = fl32(amax / 2688)          (6 * 448: the largest group scale is 448)
+ *   per token and 16-channel group g: den = fl32(s1 * 6), t = fl32(amax_g / den),
+ *   s2  = E4M3(t)  (unsigned, round to nearest even, saturating at 448)
+ *   dg  = fl32(s1 * dec(s2)),  code = E2M1(fl32(x / dg))   (0 when dg = 0)
+ * amax == 0, or s1 underflowing to 0, flushes the block (s1 = 0, every s2
+ * and code 0).  codes: [n_tok][d/2] bytes, element 2i in the low nibble;
+ * sf: [n_tok][d/16] E4M3 bytes. */
+static void quantize_block_nvfp4(const float *x, int n_tok, int d, uint8_t *codes, uint8_t *sf,
+                                 float *s1_out)
+{
+    float amax = 0.0f;
+    for (int i = 0; i < n_tok * d; i++) {
+        float a = fabsf(x[i]);
+        if (a > amax) amax = a;
+    }
+    float s1 = amax > 0.0f ? amax / 2688.0f : 0.0f;
+    for (int n = 0; n < n_tok; n++)
+        for (int g = 0; g < d / 16; g++) {
+            const float *xg = x + (size_t)n * d + 16 * g;
+            float ag = 0.0f;
+            for (int c = 0; c < 16; c++) {
+                float a = fabsf(xg[c]);
+                if (a > ag) ag = a;
+            }
+            uint8_t s2 = 0;
+            float dg = 0.0f;
+            if (s1 > 0.0f) {
+                float den = s1 * 6.0f;
+                float t = ag / den;
+                s2 = orc_e4m3_encode((double)t);
+                dg = s1 * (float)orc_e4m3_decode(s2);
+            }
+            sf[(size_t)n * (d / 16) + g] = s2;
+            for (int c = 0; c < 16; c += 2) {
+                uint8_t lo = 0, hi = 0;
+                if (dg > 0.0f) {
+                    float y0 = xg[c] / dg, y1 = xg[c + 1] / dg;
+                    lo = orc_e2m1_encode((double)y0);
+                    hi = orc_e2m1_encode((double)y1);
+                }
+                codes[(size_t)n * (d / 2) + (16 * g + c) / 2] = (uint8_t)(lo | (hi << 4));
+            }
+        }
+    *s1_out = s1;
+}
+
+/* Q and smoothed K in NVFP4 (k_mean from orc_k_mean): q4, k4 [B,H,N,d/2]
+ * packed codes; sfq, sfk [B,H,N,d/16]; sq1, sk1 [B,H,ceil(N/64)]. */
+void orc_quantize_nvfp4_qk(const uint16_t *q, const uint16_t *k, const float *k_mean,
+                           int B, int H, int N, int d, uint8_t *q4, uint8_t *k4,
+                           uint8_t *sfq, uint8_t *sfk, float *sq1, float *sk1)
+{
+    int nblk = (N + 63) / 64;
+    #pragma omp parallel for collapse(2) schedule(dynamic)
+    for (int b = 0; b < B; b++)
+        for (int h = 0; h < H; h++) {
+            float *x = (float *)malloc(sizeof(float) * 64 * d);
+            const float *mu = k_mean + ((size_t)b * H + h) * d;
+            for (int j = 0; j < nblk; j++) {
+                int nt = N - 64 * j < 64 ? N - 64 * j : 64;
+                size_t row = ((size_t)b * H + h) * N + 64 * j;
+                size_t sidx = ((size_t)b * H + h) * nblk + j;
+                for (int i = 0; i < nt * d; i++)
+                    x[i] = orc_bf16_to_float(q[row * d + i]);
+                quantize_block_nvfp4(x, nt, d, q4 + row * (d / 2), sfq + row * (d / 16), &sq1[sidx]);
+                for (int i = 0; i < nt * d; i++)
+                    x[i] = orc_bf16_to_float(k[row * d + i]) - mu[i % d];
+                quantize_block_nvfp4(x, nt, d, k4 + row * (d / 2), sfk + row * (d / 16), &sk1[sidx]);
+            }
+            free(x);
+        }
+}
+
+/* NVFP4 Q.K with the FP8 P.V path: the tiled rule of attention_core_head on
+ * the dequantized Q and K (code value x its group scale; the block scale s1
+ * plays the role of sq / sk) and the FP8 V codes and scales.  heads/rows/out
+ * as orc_attention_fp8. */
+void orc_attention_nvfp4(const uint8_t *q4, const uint8_t *k4, const uint8_t *sfq, const uint8_t *sfk,
+                         const float *sq1, const float *sk1, const uint8_t *v8, const float *sv,
+                         const float *sv_max, int B, int H, int N, int d, float softmax_scale,
+                         const int *heads, int n_heads, const int *rows, int n_rows,
+                         double *out, double *amb, int *namb)
+{
+    int nblk = (N + 63) / 64;
+    (void)B;
+    double *qc = (double *)malloc(sizeof(double) * N * d);
+    double *kc = (double *)malloc(sizeof(double) * N * d);
+    double *vc = (double *)malloc(sizeof(double) * N * d);
+    for (int hh = 0; hh < n_heads; hh++) {
+        int b = heads[2 * hh], h = heads[2 * hh + 1];
+        size_t row0 = ((size_t)b * H + h) * N;
+        for (size_t n = 0; n < (size_t)N; n++)
+            for (int c = 0; c < d; c++) {
+                size_t r = row0 + n;
+                uint8_t qb = q4[r * (d / 2) + c / 2], kb = k4[r * (d / 2) + c / 2];
+                uint8_t qn = (c & 1) ? (qb >> 4) : (qb & 15), kn = (c & 1) ? (kb >> 4) : (kb & 15);
+                qc[n * d + c] = orc_e2m1_decode(qn) * orc_e4m3_decode(sfq[r * (d / 16) + c / 16]);
+                kc[n * d + c] = orc_e2m1_decode(kn) * orc_e4m3_decode(sfk[r * (d / 16) + c / 16]);
+                vc[n * d + c] = orc_e4m3_decode(v8[r * d + c]);
+            }
+        size_t sidx = ((size_t)b * H + h) * nblk;
+        attention_core_head(qc, kc, vc, sq1 + sidx, sk1 + sidx, sv + sidx, sv_max[(size_t)b * H + h], N, d,
+                            (double)softmax_scale, 128, 1, rows, n_rows, out + (size_t)hh * n_rows * d,
+                            amb ? amb + (size_t)hh * n_rows * d : NULL,
+                            namb ? namb + (size_t)hh * n_rows : NULL, NULL, NULL, NULL);
+    }
+    free(qc); free(kc); free(vc);
+}
+
 /* --------------------------------------------- error-corrected attention */
 /* FP8 attention that corrects only the tokens with large error: "FLUX 3
  * Image Klein Base: 생성 3.46배, 8장 확장 병목", section "왜 이런 차이가 나나"
