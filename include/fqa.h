@@ -318,6 +318,56 @@ FQA_API fqa_status fqa_attention_fp8_corrected(const void* q, const void* k, con
                                                size_t workspace_bytes, void* cuda_stream);
 
 /*
+ * fqa_quantize_nvfp4_qk -- Q and smoothed K in NVFP4 for the FP4 Q.K variant.
+ * [RTX-DE] SDPA quantization paragraph: the FP8 and FP4 schemes differ only
+ * in the precision of the Q, K, V projections; attention itself stays in FP8.
+ * The element format (E2M1) and the 16-channel E4M3 group scale are the
+ * NVFP4 reading of "FP4"; V keeps its FP8 codes and scales from fqa_quantize().
+ * q, k: BF16 [B,H,N,d] (16-byte aligned); k_mean: FP32 [B,H,d], the channel
+ * means fqa_quantize() wrote for the same k.  Outputs (device, caller-owned):
+ *   q4, k4  : uint8 [B,H,N,d/2], two E2M1 codes per byte (element 2i in bits
+ *             [0,4), 2i+1 in bits [4,8)); 4-byte aligned
+ *   sfq, sfk: uint8 [B,H,N,d/16], one unsigned E4M3 scale per 16 channels
+ *   sq1, sk1: FP32 [B,H,ceil(N/64)], one scale per 64-token block
+ * Per 64-token block of x (= q, or fl32(k - k_mean) for K), in binary32:
+ *   s1 = amax / 2688 (6 x 448, so group scales reach up to 448);
+ *   per token and 16-channel group g: s2 = E4M3(amax_g / fl32(6 s1)) (round
+ *   to nearest even, saturating), dg = fl32(s1 dec(s2)),
+ *   code = E2M1(fl32(x / dg)) (nearest even, saturating to +-6; 0 if dg = 0).
+ * amax = 0 flushes the block (s1 = 0, every scale and code 0).  Any N >= 1.
+ */
+FQA_API fqa_status fqa_quantize_nvfp4_qk(const void* q, const void* k, const float* k_mean, int B, int H,
+                                         int N, int d, uint8_t* q4, uint8_t* k4, uint8_t* sfq,
+                                         uint8_t* sfk, float* sq1, float* sk1, void* cuda_stream);
+
+/*
+ * fqa_attention_nvfp4 -- attention with Q.K^T on the block-scaled FP4 tensor
+ * cores and P.V as in fqa_attention_fp8().  [RTX-DE] SDPA quantization
+ * paragraph, as fqa_quantize_nvfp4_qk().  For query row i and key j:
+ *   S_ij = sum over groups g of dec(sfq_ig) dec(sfk_jg) sum_c e2m1(q_ic) e2m1(k_jc)
+ *   x_ij = S_ij * sq1_I * sk1_J * softmax_scale * log2(e)
+ * then the fqa_attention_fp8() rule on x: exact running maximum over KV
+ * tiles of 128 keys, P = E4M3(2^(x - m) * 448 * sv_J / sv_max), O += P.V in
+ * FP32, out = O * (sv_max / 448) / l.
+ * q4 .. sk1: fqa_quantize_nvfp4_qk() outputs; v8, sv, sv_max: fqa_quantize()
+ * outputs.  q4, k4, v8 and out 16-byte aligned, sfq and sfk 8-byte aligned.
+ * N must be a multiple of 128 (FQA_ERR_UNSUPPORTED otherwise).
+ */
+FQA_API fqa_status fqa_attention_nvfp4(const uint8_t* q4, const uint8_t* k4, const uint8_t* sfq,
+                                       const uint8_t* sfk, const float* sq1, const float* sk1,
+                                       const void* v8, const float* sv, const float* sv_max, int B, int H,
+                                       int N, int d, float softmax_scale, void* out, fqa_out_dtype out_dtype,
+                                       void* cuda_stream);
+
+/*
+ * fqa_e2m1_encode -- the library's binary32 -> E2M1 conversion (round to
+ * nearest even, saturating to +-6), two values per byte as in
+ * fqa_quantize_nvfp4_qk: out[i] = code(x[2i]) | code(x[2i+1]) << 4.
+ * x: FP32 [2 npairs], 8-byte aligned; out: uint8 [npairs] (device).
+ */
+FQA_API fqa_status fqa_e2m1_encode(const float* x, uint8_t* out, size_t npairs, void* cuda_stream);
+
+/*
  * fqa_e4m3_encode -- the library's binary32 -> E4M3 conversion (round to
  * nearest even, saturating to +-448, NaN -> 0x7F), exposed so that callers
  * can check the codec exhaustively.  x: FP32 [n], out: uint8 [n] (device).

@@ -69,6 +69,12 @@ def _load():
     L.fqa_attention_fp8_corrected.restype = I
     L.fqa_attention_fp8_corrected.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, I, I, I, I, ctypes.c_float,
                                               ctypes.c_float, P, I, P, ctypes.c_size_t, P]
+    L.fqa_quantize_nvfp4_qk.restype = I
+    L.fqa_quantize_nvfp4_qk.argtypes = [P, P, P, I, I, I, I, P, P, P, P, P, P, P]
+    L.fqa_attention_nvfp4.restype = I
+    L.fqa_attention_nvfp4.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, ctypes.c_float, P, I, P]
+    L.fqa_e2m1_encode.restype = I
+    L.fqa_e2m1_encode.argtypes = [P, P, ctypes.c_size_t, P]
     _lib = L
     return L
 
@@ -200,6 +206,24 @@ def fqa_attention_fp8_corrected(q, k, v, q8, k8, v8, sq, sk, sv, sv_max, k_mean,
 
 def fqa_e4m3_encode(x, out, stream=None) -> int:
     return _load().fqa_e4m3_encode(_ptr(x), _ptr(out), x.numel(), _stream(stream))
+
+
+def fqa_quantize_nvfp4_qk(q, k, k_mean, q4, k4, sfq, sfk, sq1, sk1, stream=None) -> int:
+    B, H, N, d = q.shape
+    return _load().fqa_quantize_nvfp4_qk(_ptr(q), _ptr(k), _ptr(k_mean), B, H, N, d, _ptr(q4), _ptr(k4),
+                                         _ptr(sfq), _ptr(sfk), _ptr(sq1), _ptr(sk1), _stream(stream))
+
+
+def fqa_attention_nvfp4(q4, k4, sfq, sfk, sq1, sk1, v8, sv, sv_max, softmax_scale, out, out_dtype,
+                        stream=None) -> int:
+    B, H, N, d = v8.shape
+    return _load().fqa_attention_nvfp4(_ptr(q4), _ptr(k4), _ptr(sfq), _ptr(sfk), _ptr(sq1), _ptr(sk1), _ptr(v8),
+                                       _ptr(sv), _ptr(sv_max), B, H, N, d, float(softmax_scale), _ptr(out),
+                                       int(out_dtype), _stream(stream))
+
+
+def fqa_e2m1_encode(x, out, stream=None) -> int:
+    return _load().fqa_e2m1_encode(_ptr(x), _ptr(out), x.numel() // 2, _stream(stream))
 
 
 def fqa_debug_wait_timeout(limit_us: int, stream=None) -> int:
@@ -418,6 +442,82 @@ def e4m3_encode(x: torch.Tensor, stream=None) -> torch.Tensor:
     _require(x, torch.float32, "x")
     out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
     _check(fqa_e4m3_encode(x, out, stream=stream), "fqa_e4m3_encode")
+    return out
+
+
+# ------------------------------------------------ NVFP4 Q.K variant
+
+class QuantizedNvfp4(NamedTuple):
+    q4: torch.Tensor       # uint8 [B,H,N,64]: E2M1 codes, element 2i in the low nibble
+    k4: torch.Tensor       # of K - k_mean
+    sfq: torch.Tensor      # uint8 [B,H,N,8]: E4M3 scale per 16 channels
+    sfk: torch.Tensor
+    sq1: torch.Tensor      # float32 [B,H,ceil(N/64)]
+    sk1: torch.Tensor
+
+
+def alloc_quantized_nvfp4(B: int, H: int, N: int, device) -> QuantizedNvfp4:
+    u8 = dict(dtype=torch.uint8, device=device)
+    f32 = dict(dtype=torch.float32, device=device)
+    nb = nblocks(N)
+    return QuantizedNvfp4(torch.empty(B, H, N, HEAD_DIM // 2, **u8), torch.empty(B, H, N, HEAD_DIM // 2, **u8),
+                          torch.empty(B, H, N, HEAD_DIM // 16, **u8), torch.empty(B, H, N, HEAD_DIM // 16, **u8),
+                          torch.empty(B, H, nb, **f32), torch.empty(B, H, nb, **f32))
+
+
+def _require_nvfp4(qn: QuantizedNvfp4, B: int, H: int, N: int) -> None:
+    nb = nblocks(N)
+    shapes = ((B, H, N, HEAD_DIM // 2),) * 2 + ((B, H, N, HEAD_DIM // 16),) * 2 + ((B, H, nb),) * 2
+    for name, t, shape in zip(QuantizedNvfp4._fields, qn, shapes):
+        _require(t, torch.float32 if name.endswith("1") else torch.uint8, name, shape)
+
+
+def quantize_nvfp4_qk(q: torch.Tensor, k: torch.Tensor, k_mean: torch.Tensor,
+                      out: Optional[QuantizedNvfp4] = None, stream=None) -> QuantizedNvfp4:
+    """BF16 Q, K [B,H,N,128] and the K channel means of quantize() -> NVFP4 Q and
+    smoothed K."""
+    B, H, N, _ = _require_qkv(q, k, k, torch.bfloat16)
+    _require(k_mean, torch.float32, "k_mean", (B, H, HEAD_DIM))
+    if out is None:
+        out = alloc_quantized_nvfp4(B, H, N, q.device)
+    _require_nvfp4(out, B, H, N)
+    _check(fqa_quantize_nvfp4_qk(q, k, k_mean, *out, stream=stream), "fqa_quantize_nvfp4_qk")
+    return out
+
+
+def attention_nvfp4(qn: QuantizedNvfp4, qz: Quantized, softmax_scale: float, out_dtype: int = FQA_OUT_BF16,
+                    out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """NVFP4 Q.K^T, FP8 P.V: qn from quantize_nvfp4_qk(), V (v8, sv, sv_max) from qz."""
+    if not isinstance(qz.v8, torch.Tensor) or qz.v8.dim() != 4:
+        raise ValueError("qz.v8: expected a [B, H, N, 128] tensor")
+    B, H, N, d = qz.v8.shape
+    _require_quantized(qz, B, H, N)
+    _require_nvfp4(qn, B, H, N)
+    dt = torch.float32 if out_dtype == FQA_OUT_F32 else torch.bfloat16
+    if out is None:
+        out = torch.empty(B, H, N, d, dtype=dt, device=qz.v8.device)
+    _require(out, dt, "out", (B, H, N, d))
+    _check(fqa_attention_nvfp4(*qn, qz.v8, qz.sv, qz.sv_max, softmax_scale, out, out_dtype, stream=stream),
+           "fqa_attention_nvfp4")
+    return out
+
+
+def nvfp4_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, softmax_scale: float,
+                    out_dtype: int = FQA_OUT_BF16, stream=None) -> torch.Tensor:
+    """The whole FP4 Q.K path: quantize (V codes and the K mean), NVFP4 Q and
+    K, then the attention."""
+    qz = quantize(q, k, v, stream=stream)
+    return attention_nvfp4(quantize_nvfp4_qk(q, k, qz.k_mean, stream=stream), qz, softmax_scale, out_dtype,
+                           stream=stream)
+
+
+def e2m1_encode(x: torch.Tensor, stream=None) -> torch.Tensor:
+    """FP32 [..., 2n] -> uint8 [..., n]: two E2M1 codes per byte, x[2i] in the low nibble."""
+    _require(x, torch.float32, "x")
+    if x.numel() % 2:
+        raise ValueError("x: expected an even number of elements")
+    out = torch.empty(x.numel() // 2, dtype=torch.uint8, device=x.device)
+    _check(fqa_e2m1_encode(x, out, stream=stream), "fqa_e2m1_encode")
     return out
 
 

@@ -547,7 +547,6 @@ __global__ void __launch_bounds__(kF8Threads, 1)
       if constexpr (kMaskable) {
         if (p.row_stats != nullptr && hf == 0 && store) p.row_stats[orow] = make_float2(m, l_row);
       }
-#pragma unroll 1
       // the output row: [B,H,N,128], or with out_P > 1 the sequence all-to-all
       // layout [B, out_P, H, N / out_P, 128] (chunk c: tokens [c N/out_P, ...))
       size_t orow_out = orow;
@@ -555,6 +554,7 @@ __global__ void __launch_bounds__(kF8Threads, 1)
         const int nl = N / p.out_P, cq = qrow / nl;
         orow_out = (((size_t)w.b * p.out_P + cq) * p.H + w.h) * nl + (qrow - cq * nl);
       }
+#pragma unroll 1
       for (int c = 0; c < 2; ++c) {
         uint32_t o[32];
         const int col = 64 * hf + 32 * c;

@@ -304,6 +304,16 @@ __device__ __forceinline__ uint32_t e4m3x4(float v0, float v1, float v2, float v
   return d;
 }
 
+// Two binary32 values -> two E2M1 codes (round to nearest even, saturating
+// to +-6) in one byte: `lo` in bits [0,4), `hi` in bits [4,8).
+__device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 c;\n\tcvt.rn.satfinite.e2m1x2.f32 c, %1, %2;\n\tcvt.u32.u8 %0, c;\n\t}"
+      : "=r"(r)
+      : "f"(hi), "f"(lo));
+  return r;
+}
+
 // Two E4M3 codes (bits [0,8) and [8,16)) -> their exact binary32 values.
 __device__ __forceinline__ float2 e4m3x2_to_f2(uint32_t codes) {
   uint32_t h2;

@@ -12,10 +12,12 @@
 #include "../../include/fqa.h"
 #include "attention.cuh"
 #include "attention_fp8.cuh"
+#include "attention_nvfp4.cuh"
 #include "attention_ws.cuh"
 #include "correct.cuh"
 #include "device.cuh"
 #include "quantize.cuh"
+#include "quantize_nvfp4.cuh"
 
 namespace fqa {
 
@@ -89,6 +91,22 @@ static bool make_tmap(CUtensorMap* m, const void* base, bool fp8, int N, int hea
   CUresult r = enc(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
                    const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// 3-D view (byte, row within the head, head) of packed E2M1 codes
+// [B,H,N,64 B]; box = 64 B x 128 rows x 1 head, 64-byte swizzle (the layout
+// the block-scaled MMA reads through a SWIZZLE_64B descriptor).
+static bool make_tmap_fp4(CUtensorMap* m, const void* base, int N, int heads) {
+  EncodeTiledFn enc = encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {64, (cuuint64_t)N, (cuuint64_t)heads};
+  cuuint64_t strides[2] = {64ull, 64ull * (cuuint64_t)N};
+  cuuint32_t box[3] = {64u, 128u, 1u};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -463,6 +481,72 @@ fqa_status fqa_attention_fp8_corrected(const void* q, const void* k, const void*
   if (split > ntq) split = ntq;
   if (split < 1) split = 1;
   correct_kernel<<<dim3(split, B * H), kCorrThreads, CorrTraits::kSmemBytes, s>>>(tq, cp);
+  return launch_status();
+}
+
+// ------------------------------------------------------- NVFP4 Q.K variant
+
+fqa_status fqa_quantize_nvfp4_qk(const void* q, const void* k, const float* k_mean, int B, int H, int N, int d,
+                                 uint8_t* q4, uint8_t* k4, uint8_t* sfq, uint8_t* sfk, float* sq1, float* sk1,
+                                 void* cuda_stream) {
+  fqa_status st = check_shape(B, H, N, d);
+  if (st != FQA_OK) return st;
+  const void* ptrs[] = {q, k, k_mean, q4, k4, sfq, sfk, sq1, sk1};
+  for (const void* p : ptrs)
+    if (p == nullptr) return FQA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16)) return FQA_ERR_MISALIGNED;
+  const void* a4[] = {k_mean, q4, k4, sq1, sk1};
+  for (const void* p : a4)
+    if (!aligned(p, 4)) return FQA_ERR_MISALIGNED;
+  const int units = B * H * ((N + 63) / 64);
+  quantize_nvfp4_kernel<<<2 * units, kNv4Threads, 0, static_cast<cudaStream_t>(cuda_stream)>>>(
+      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), k_mean, q4, k4, sfq, sfk,
+      sq1, sk1, B, H, N);
+  return launch_status();
+}
+
+fqa_status fqa_attention_nvfp4(const uint8_t* q4, const uint8_t* k4, const uint8_t* sfq, const uint8_t* sfk,
+                               const float* sq1, const float* sk1, const void* v8, const float* sv,
+                               const float* sv_max, int B, int H, int N, int d, float softmax_scale, void* out,
+                               fqa_out_dtype out_dtype, void* cuda_stream) {
+  fqa_status st = check_attention_common(B, H, N, d, softmax_scale, out, out_dtype);
+  if (st != FQA_OK) return st;
+  if (N % kBlockN != 0) return FQA_ERR_UNSUPPORTED;
+  const void* ptrs[] = {q4, k4, sfq, sfk, sq1, sk1, v8, sv, sv_max};
+  for (const void* p : ptrs)
+    if (p == nullptr) return FQA_ERR_INVALID_ARG;
+  const void* a16[] = {q4, k4, v8};
+  for (const void* p : a16)
+    if (!aligned(p, 16)) return FQA_ERR_MISALIGNED;
+  if (!aligned(sfq, 8) || !aligned(sfk, 8)) return FQA_ERR_MISALIGNED;
+  const void* a4[] = {sq1, sk1, sv, sv_max};
+  for (const void* p : a4)
+    if (!aligned(p, 4)) return FQA_ERR_MISALIGNED;
+  uint32_t* status = status_ptr(&st);
+  if (!status) return st;
+  const int heads = B * H;
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap_fp4(&tq, q4, N, heads) || !make_tmap_fp4(&tk, k4, N, heads) ||
+      !make_tmap(&tv, v8, true, N, heads))
+    return FQA_ERR_CUDA;
+  if (cudaFuncSetAttribute(attn_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           NvTraits::kSmemBytes) != cudaSuccess)
+    return FQA_ERR_CUDA;
+  NvParams prm{B, H, N, softmax_scale, sfq, sfk, sq1, sk1, sv, sv_max, out, out_dtype == FQA_OUT_F32, status};
+  const int items = heads * (N / kBlockM);
+  const int sms = num_sms();
+  if (sms <= 0) return FQA_ERR_CUDA;
+  const int grid = items < sms ? items : sms;
+  attn_nvfp4_kernel<<<grid, kNvThreads, NvTraits::kSmemBytes, static_cast<cudaStream_t>(cuda_stream)>>>(
+      tq, tk, tv, prm);
+  return launch_status();
+}
+
+fqa_status fqa_e2m1_encode(const float* x, uint8_t* out, size_t npairs, void* cuda_stream) {
+  if (x == nullptr || out == nullptr) return FQA_ERR_INVALID_ARG;
+  if (npairs == 0) return FQA_OK;
+  if (!aligned(x, 8)) return FQA_ERR_MISALIGNED;
+  e2m1_encode_kernel<<<148 * 8, 256, 0, static_cast<cudaStream_t>(cuda_stream)>>>(x, out, npairs);
   return launch_status();
 }
 

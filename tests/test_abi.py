@@ -128,3 +128,39 @@ def test_corrected_key_count_matches_the_oracle(L):
     assert fqa.fqa_corrected_keys(100, float("nan")) == -1
     assert fqa.fqa_attention_fp8_corrected_workspace_bytes(1, 24, 8704, 0.005) > 24 * 8704 * 512
     assert fqa.fqa_attention_fp8_corrected_workspace_bytes(1, 24, 8704, 2.0) == 0
+
+
+def test_nvfp4_validation(L):
+    ok = _p(0x10000)
+    f = ctypes.c_float
+
+    def quant(**kw):
+        return L.fqa_quantize_nvfp4_qk(kw.get("q", ok), kw.get("k", ok), kw.get("km", ok), kw.get("B", 1),
+                                       kw.get("H", 1), kw.get("N", 128), kw.get("d", 128),
+                                       *[kw.get(n, ok) for n in ("q4", "k4", "sfq", "sfk", "sq1", "sk1")], None)
+
+    def attn(**kw):
+        return L.fqa_attention_nvfp4(*[kw.get(n, ok) for n in ("q4", "k4", "sfq", "sfk", "sq1", "sk1", "v8",
+                                                                "sv", "svm")],
+                                     kw.get("B", 1), kw.get("H", 1), kw.get("N", 128), kw.get("d", 128),
+                                     f(kw.get("scale", 0.088)), kw.get("out", ok), kw.get("dt", 0), None)
+
+    assert quant(q=None) == 1
+    assert quant(sk1=None) == 1
+    assert quant(N=0) == 1
+    assert quant(d=64) == 2
+    assert quant(N=65537) == 2
+    assert quant(k=_p(0x10008)) == 3            # BF16 inputs: 16-byte aligned
+    assert quant(q4=_p(0x10002)) == 3           # packed codes: 4-byte aligned
+    assert attn(q4=None) == 1
+    assert attn(out=None) == 1
+    assert attn(scale=0.0) == 1
+    assert attn(dt=3) == 1
+    assert attn(N=200) == 2                     # N must be a multiple of 128
+    assert attn(N=65537) == 2
+    assert attn(d=64) == 2
+    assert attn(k4=_p(0x10008)) == 3
+    assert attn(sfq=_p(0x10004)) == 3           # group scales: 8-byte aligned
+    assert attn(sv=_p(0x10002)) == 3
+    assert L.fqa_e2m1_encode(None, ok, 4, None) == 1
+    assert L.fqa_e2m1_encode(_p(0x10004), ok, 4, None) == 3
