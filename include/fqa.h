@@ -123,10 +123,11 @@ FQA_API size_t fqa_quantize_workspace_bytes(int B, int H, int N, int d);
  * k_mean       out: FP32 [B,H,d]
  * workspace    scratch of at least fqa_quantize_workspace_bytes(B,H,N,d)
  *              bytes, 16-byte aligned; contents on entry are ignored.
- * Enqueues on cuda_stream a 16-byte memset of the workspace counters and one
- * cooperative kernel launch (Q/V codes and K partial sums; K mean and V head
- * maxima; K codes -- phases separated by bounded grid barriers, 64-token
- * blocks handed out through work queues).
+ * Enqueues on cuda_stream a 24-byte memset of the workspace counters and one
+ * cooperative kernel launch (V codes and K partial sums; K mean and V head
+ * maxima; K codes -- phases separated by bounded grid barriers, with the Q
+ * codes computed while each barrier completes; 64-token blocks handed out
+ * through work queues).
  */
 FQA_API fqa_status fqa_quantize(const void* q, const void* k, const void* v, int B, int H, int N, int d,
                         void* q8, void* k8, void* v8, float* sq, float* sk, float* sv,

@@ -20,6 +20,8 @@
 // Inputs are BF16 [B,H,N,128]; codes are written in the same layout.
 #pragma once
 
+#include <type_traits>
+
 #include "device.cuh"
 
 namespace fqa {
@@ -27,13 +29,17 @@ namespace fqa {
 // ---------------------------------------------------------------------------
 // Fused quantizer: one cooperative persistent launch in three phases separated
 // by grid barriers (the K codes need the K mean, which needs all of K):
-//   1a  Q and V units -> codes and scales
-//   1b  K units -> per-unit partial sums (per channel, 64 tokens in order);
-//       K read last and marked evict-last in L2 for phase 3
+//   1   V units -> codes and scales; then K units -> per-unit partial sums
+//       (per channel, 64 tokens in order), K marked evict-last in L2 for 3
 //   2   per (b, h): k_mean from the partials in block order; sv_max = max of
 //       the V unit scales (no atomics)
-//   3   K units -> smoothed codes and scales, newest units of 1b first (each
+//   3   K units -> smoothed codes and scales, newest units of 1 first (each
 //       unit's head mean row arrives with the unit)
+// Q is needed by none of the phases, so its units fill the barrier waits:
+// each barrier is split into an arrival and a wait, and the first half of
+// the Q units runs between the arrival and the wait of barrier 1, the second
+// half between those of barrier 2 (while other SMs finish their K units, and
+// while phase 2 runs), keeping HBM busy through both.
 // Unit u = (b*H + h)*ceil(N/64) + j is one 64-token block of one head: 16 KB
 // of contiguous BF16 per tensor (the last block of a head may be shorter).  Units are handed out through work queues
 // (counters the launch zeroes), so the SMs that stream faster take more.
@@ -47,31 +53,40 @@ constexpr int kQuantWarps = kQuantThreads / 32;
 constexpr int kBlockBytes = kQBlock * kHeadDim * 2;            // 16 KB of BF16
 constexpr int kChunks = kBlockBytes / 16 / kQuantThreads;       // 16-byte chunks per thread
 constexpr int kVals = 8 * kChunks;
-constexpr int kRingBytes = 64 * 1024;             // three CTAs per SM
+constexpr int kRingBytes = 48 * 1024;             // four CTAs per SM
 constexpr int kMaxSlots = kRingBytes / kBlockBytes;
 constexpr int kQuantSmem = kRingBytes + 128;
 constexpr int kPartialRowsPerSlot = kBlockBytes / (kHeadDim * 4);   // 32 partial rows per 16 KB
 // CTAs the shared memory admits per SM (the register cap follows from it)
-constexpr int kQuantMinCtas = (200 * 1024) / (kQuantSmem + 2048) < 1 ? 1 : (200 * 1024) / (kQuantSmem + 2048);
-static_assert(kMaxSlots >= 4 && kMaxSlots <= 32, "ring size");
+constexpr int kQuantMinCtas = (228 * 1024) / (kQuantSmem + 2048) < 1 ? 1 : (228 * 1024) / (kQuantSmem + 2048);
+static_assert(kMaxSlots >= 3 && kMaxSlots <= 32, "ring size");
+static_assert(kRingBytes / (kBlockBytes + kHeadDim * 4) >= 2, "two slots in every pass");
 static_assert(kQuantThreads >= 2 * kHeadDim, "k_mean and sv_max threads");
 static_assert((kQuantThreads * 8) % kHeadDim == 0, "chunk c of thread t starts at channel 8t mod 128");
 
 // Counters the launch zeroes (in the workspace, after the partial sums).
 constexpr int kCtrBarrier = 0;     // grid barrier arrivals
-constexpr int kCtrQV = 1;          // next unit of phase 1a
-constexpr int kCtrK = 2;           // next unit of phase 1b
+constexpr int kCtrV = 1;           // next V unit (phase 1)
+constexpr int kCtrK = 2;           // next K unit of phase 1
 constexpr int kCtrK3 = 3;          // next unit of phase 3 (counted from the end)
-constexpr int kNumCtr = 4;
+constexpr int kCtrQA = 4;          // next Q unit of the first half
+constexpr int kCtrQB = 5;          // next Q unit of the second half
+constexpr int kNumCtr = 6;
 
-// Grid barrier number `round` (1, 2, ...): arrive, then wait until every CTA
-// of the grid has arrived `round` times.  Gives up after kWaitLimitNs.
-__device__ __forceinline__ bool grid_barrier(unsigned int* ctr, unsigned int round, uint32_t* status,
-                                             volatile int* failed) {
+// Grid barrier, split: grid_arrive() publishes this CTA's earlier writes and
+// counts it in; grid_wait(round) waits until every CTA of the grid has
+// arrived `round` times (round 1, 2, ...), giving up after kWaitLimitNs.
+// Work between the two calls is not covered by the barrier.
+__device__ __forceinline__ void grid_arrive(unsigned int* ctr) {
   __syncthreads();
   if (threadIdx.x == 0) {
     __threadfence();
     atomicAdd(ctr, 1u);
+  }
+}
+__device__ __forceinline__ bool grid_wait(unsigned int* ctr, unsigned int round, uint32_t* status,
+                                          volatile int* failed) {
+  if (threadIdx.x == 0) {
     const unsigned int target = round * gridDim.x;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
@@ -125,12 +140,17 @@ __device__ __forceinline__ float residual_sq8(const float* x, const uint32_t (&w
   return acc;
 }
 
-// Block absmax over the CTA (red: one float per warp for this slot), scale,
-// and the codes of this thread's chunks (8 bytes per chunk, chunk c at byte
-// 8c; chunks at or beyond nvalid are not stored).  rsq (optional): each
-// chunk's residual squares (residual_sq8).
-__device__ __forceinline__ float quantize_chunks(float (&x)[kVals], float* red, uint8_t* dst, int slot,
-                                                 int nvalid, uint64_t policy, float* rsq = nullptr) {
+// Block absmax over the CTA (red: one float per warp, in buffer `slot`),
+// scale, and the codes of this thread's chunks (8 bytes per chunk, chunk c at
+// byte 8c; chunks at or beyond nvalid are not stored).  The CTA-wide sync of
+// the absmax also combines `ok` (this thread's wait for the unit): unless
+// every thread's is true nothing is stored and false is returned.  It is the
+// unit's one sync: the caller's slot may be refilled after it (x holds the
+// values) and the other `red` buffer is free for the next unit.  rsq
+// (optional): each chunk's residual squares (residual_sq8).
+__device__ __forceinline__ bool quantize_chunks(float (&x)[kVals], float* red, uint8_t* dst, int slot,
+                                                int nvalid, uint64_t policy, bool ok, float& scale_out,
+                                                float* rsq = nullptr) {
   const int t = threadIdx.x;
   float m = 0.0f;
 #pragma unroll
@@ -138,7 +158,7 @@ __device__ __forceinline__ float quantize_chunks(float (&x)[kVals], float* red, 
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   if ((t & 31) == 0) red[slot * kQuantWarps + (t >> 5)] = m;
-  __syncthreads();
+  if (!__syncthreads_and(ok)) return false;
   float a = red[slot * kQuantWarps];
 #pragma unroll
   for (int w = 1; w < kQuantWarps; ++w) a = fmaxf(a, red[slot * kQuantWarps + w]);
@@ -158,7 +178,8 @@ __device__ __forceinline__ float quantize_chunks(float (&x)[kVals], float* red, 
         st_global_v2_hint(dst + 8 * (t + kQuantThreads * i), w[0] | (w[1] << 16), w[2] | (w[3] << 16), policy);
       if (rsq) rsq[i] = residual_sq8(&x[8 * i], w, scale);
     }
-    return scale;
+    scale_out = scale;
+    return true;
   }
 #pragma unroll
   for (int i = 0; i < kChunks; ++i) {
@@ -173,7 +194,8 @@ __device__ __forceinline__ float quantize_chunks(float (&x)[kVals], float* red, 
       rsq[i] = residual_sq8(&x[8 * i], w, scale);
     }
   }
-  return scale;
+  scale_out = scale;
+  return true;
 }
 
 __global__ void __launch_bounds__(kQuantThreads, kQuantMinCtas) quantize_fused_kernel(
@@ -207,11 +229,18 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantMinCtas) quantize_fused_k
   // One pipelined pass with slots of slot_bytes.  next() (thread 0) yields
   // the next unit index, or -1 when there is none and from then on;
   // issue(u, dst, bar) starts unit u's bulk copies (it arms bar itself);
-  // body(u, slot memory) runs on all threads, in the order next() gave the
-  // units.  Every started copy is waited for before the pass returns, unless
-  // a wait timed out (returns false).
+  // body(u, slot memory, ok, parity) runs on all threads, in the order next()
+  // gave the units, ok being this thread's wait for the unit and parity the
+  // unit's count mod 2.  A body that returns bool contains one
+  // __syncthreads_and(ok) after its last read of the slot (the slot is then
+  // refilled while the body finishes) and returns its result; any other body
+  // is fenced by syncs on both sides.  Every started copy is waited for
+  // before the pass returns, unless a wait timed out (returns false).
   auto run = [&](int slot_bytes, auto next, auto issue, auto body) -> bool {
     const int nslots = kRingBytes / slot_bytes;
+    // every thread has left the previous pass (a body-synced pass ends with
+    // threads past their last sync but not yet at the loop's exit test)
+    __syncthreads();
     if (t == 0)
       for (int s = 0; s < nslots - 1; ++s) {
         const int u = next();
@@ -219,6 +248,7 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantMinCtas) quantize_fused_k
         if (u >= 0) issue(u, ring + s * slot_bytes, &full[s]);
       }
     __syncthreads();
+    int it = 0;
     for (int s = 0;; s = (s + 1 == nslots) ? 0 : s + 1) {
       const int u = slot_unit[s];
       if (u < 0) break;                            // CTA-uniform
@@ -231,23 +261,29 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantMinCtas) quantize_fused_k
       }
       const bool ok = mbar_wait(&full[s], (phase_bits >> s) & 1u, &abort_flag, status);
       phase_bits ^= 1u << s;
-      if (!__syncthreads_and(ok)) return false;
-      body(u, ring + s * slot_bytes);
-      __syncthreads();                             // slot s, slot_unit and red free again
+      using R = decltype(body(u, ring, ok, 0));
+      if constexpr (std::is_same<R, bool>::value) {
+        if (!body(u, ring + s * slot_bytes, ok, it & 1)) return false;
+      } else {
+        if (!__syncthreads_and(ok)) return false;
+        body(u, ring + s * slot_bytes, ok, it & 1);
+        __syncthreads();                           // slot s and slot_unit free again
+      }
+      ++it;
     }
     return true;
   };
-  // a shared work queue over all units: ctr[c] counts the units handed out
-  auto queue = [&](int c, bool reverse) {
+  // a shared work queue over units [lo, hi): ctr[c] counts the units handed out
+  auto queue = [&](int c, int lo, int hi, bool reverse) {
     bool drained = false;
     return [=]() mutable -> int {
       if (drained) return -1;
       const unsigned int i = atomicAdd(&ctr[c], 1u);
-      if (i >= (unsigned int)nunits) {
+      if (i >= (unsigned int)(hi - lo)) {
         drained = true;
         return -1;
       }
-      return reverse ? nunits - 1 - (int)i : (int)i;
+      return reverse ? hi - 1 - (int)i : lo + (int)i;
     };
   };
   // element offset of unit u in a [B,H,N,128] tensor (the codes, and the
@@ -270,37 +306,37 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantMinCtas) quantize_fused_k
   };
   auto unit_rows = [&](int u) { return min(kQBlock, N - (u % nblk) * kQBlock); };
 
-  // ---- phase 1a: Q and V (streamed once: evict-first)
-  bool ok = run(2 * kBlockBytes, queue(kCtrQV, false),
-      [&](int u, uint8_t* dst, uint64_t* bar) {
-        const uint32_t bytes = (uint32_t)unit_rows(u) * kHeadDim * 2;
-        mbar_arrive_expect_tx(bar, 2 * bytes);
-        bulk_load(dst, q + unit_in(u), bytes, bar, pol_first);
-        bulk_load(dst + kBlockBytes, v + unit_in(u), bytes, bar, pol_first);
-      },
-      [&](int u, const uint8_t* blk) {
-        const size_t off = unit_off(u);
-        const int nvalid = unit_rows(u) * (kHeadDim * 2 / 16);
-        float x[kVals];
-        chunks_to_f32(blk, nvalid, x);
-        const float s_q = quantize_chunks(x, red, q8 + off, 0, nvalid, pol_first);
-        chunks_to_f32(blk + kBlockBytes, nvalid, x);
-        const float s_v = quantize_chunks(x, red, v8 + off, 1, nvalid, pol_first);
-        if (t == 0) {
-          sq[u] = s_q;
-          sv[u] = s_v;
-        }
-      });
-  // ---- phase 1b: K partial sums (one thread per channel adds the unit's 64
-  // tokens in order); K stays in L2 for phase 3
+  // Q or V units (streamed once: evict-first) -> codes and block scales
+  auto pass_qv = [&](const __nv_bfloat16* src, uint8_t* codes, float* scales, auto next) -> bool {
+    return run(kBlockBytes, next,
+        [&](int u, uint8_t* dst, uint64_t* bar) {
+          const uint32_t bytes = (uint32_t)unit_rows(u) * kHeadDim * 2;
+          mbar_arrive_expect_tx(bar, bytes);
+          bulk_load(dst, src + unit_in(u), bytes, bar, pol_first);
+        },
+        [&](int u, const uint8_t* blk, bool ok, int par) -> bool {
+          const int nvalid = unit_rows(u) * (kHeadDim * 2 / 16);
+          float x[kVals];
+          chunks_to_f32(blk, nvalid, x);
+          float sc;
+          if (!quantize_chunks(x, red, codes + unit_off(u), par, nvalid, pol_first, ok, sc)) return false;
+          if (t == 0) scales[u] = sc;
+          return true;
+        });
+  };
+  const int nqa = (nunits + 1) / 2;                // Q units before barrier 1's wait
+
+  // ---- phase 1: V, then the K partial sums (one thread per channel adds the
+  // unit's 64 tokens in order); K stays in L2 for phase 3
+  bool ok = pass_qv(v, v8, sv, queue(kCtrV, 0, nunits, false));
   if (ok)
-    ok = run(kBlockBytes, queue(kCtrK, false),
+    ok = run(kBlockBytes, queue(kCtrK, 0, nunits, false),
         [&](int u, uint8_t* dst, uint64_t* bar) {
           const uint32_t bytes = (uint32_t)unit_rows(u) * kHeadDim * 2;
           mbar_arrive_expect_tx(bar, bytes);
           bulk_load(dst, k + unit_in(u), bytes, bar, pol_last);
         },
-        [&](int u, const uint8_t* blk) {
+        [&](int u, const uint8_t* blk, bool, int) {
           if (t < kHeadDim) {
             const __nv_bfloat16* kb = reinterpret_cast<const __nv_bfloat16*>(blk);
             const int rows = unit_rows(u);
@@ -315,7 +351,10 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantMinCtas) quantize_fused_k
           }
         });
   if (!ok) failed = 1;
-  if (!grid_barrier(&ctr[kCtrBarrier], 1, status, &failed)) return;
+  grid_arrive(&ctr[kCtrBarrier]);
+  // the first half of Q while the other SMs finish phase 1
+  if (ok && !pass_qv(q, q8, sq, queue(kCtrQA, 0, nqa, false))) failed = 1;
+  if (!grid_wait(&ctr[kCtrBarrier], 1, status, &failed)) return;
 
   // ---- phase 2: per (b, h), k_mean (threads 0..127: one channel each, the
   // partials staged 32 rows a slot and added in block order) and sv_max
@@ -340,7 +379,7 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantMinCtas) quantize_fused_k
           bulk_load(dst, src + (size_t)i * kPartialRowsPerSlot * kHeadDim, rows * kHeadDim * 4, bar,
                     pol_first);
         },
-        [&](int i, const uint8_t* blk) {
+        [&](int i, const uint8_t* blk, bool, int) {
           if (t < kHeadDim) {
             const float* pr = reinterpret_cast<const float*>(blk);
             const int rows = min(kPartialRowsPerSlot, nblk - i * kPartialRowsPerSlot);
@@ -361,19 +400,22 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantMinCtas) quantize_fused_k
     }
     __syncthreads();                               // red reused by the next head
   }
-  if (!grid_barrier(&ctr[kCtrBarrier], 2, status, &failed)) return;
+  grid_arrive(&ctr[kCtrBarrier]);
+  // the second half of Q while phase 2 completes on the other SMs
+  if (!failed && !pass_qv(q, q8, sq, queue(kCtrQB, nqa, nunits, false))) failed = 1;
+  if (!grid_wait(&ctr[kCtrBarrier], 2, status, &failed)) return;
 
   // ---- phase 3: K codes, newest units of phase 1b first.  Each slot holds
   // the unit's K block and its head's k_mean row (512 B), loaded together.
   constexpr int kSlot3 = kBlockBytes + kHeadDim * 4;
-  run(kSlot3, queue(kCtrK3, true),
+  run(kSlot3, queue(kCtrK3, 0, nunits, true),
       [&](int u, uint8_t* dst, uint64_t* bar) {
         const uint32_t bytes = (uint32_t)unit_rows(u) * kHeadDim * 2;
         mbar_arrive_expect_tx(bar, bytes + kHeadDim * 4);
         bulk_load(dst, k + unit_in(u), bytes, bar, pol_first);
         bulk_load(dst + kBlockBytes, k_mean + (size_t)(u / nblk) * kHeadDim, kHeadDim * 4, bar, pol_first);
       },
-      [&](int u, const uint8_t* blk) {
+      [&](int u, const uint8_t* blk, bool ok, int par) -> bool {
         // every chunk of this thread starts at channel 8t mod 128
         const float* mu = reinterpret_cast<const float*>(blk + kBlockBytes) + ((8 * t) & (kHeadDim - 1));
         float mr[8];
@@ -390,17 +432,18 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantMinCtas) quantize_fused_k
             for (int e = 0; e < 8; ++e) x[8 * i4 + e] = __fsub_rn(x[8 * i4 + e], mr[e]);
           }
         }
+        float s_k;
         if (k_err == nullptr) {
-          const float s_k = quantize_chunks(x, red, k8 + unit_off(u), 0, nvalid, pol_first);
+          if (!quantize_chunks(x, red, k8 + unit_off(u), par, nvalid, pol_first, ok, s_k)) return false;
           if (t == 0) sk[u] = s_k;
-          return;
+          return true;
         }
         // with the per-key quantization error: chunk i of this thread is
         // channels 8 (t % 16) .. +8 of token t / 16 + 16 i of the unit; the 16
         // lanes of a token combine their chunk sums pairwise in the pinned
         // order g_l + g_l^8, then ^4, ^2, ^1 (identical in every lane)
         float rsq[kChunks];
-        const float s_k = quantize_chunks(x, red, k8 + unit_off(u), 0, nvalid, pol_first, rsq);
+        if (!quantize_chunks(x, red, k8 + unit_off(u), par, nvalid, pol_first, ok, s_k, rsq)) return false;
         if (t == 0) sk[u] = s_k;
         const size_t tok0 = unit_off(u) / kHeadDim;
 #pragma unroll
@@ -413,6 +456,7 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantMinCtas) quantize_fused_k
           const int c = t + kQuantThreads * i;
           if ((t & 15) == 0 && c < nvalid) k_err[tok0 + c / 16] = e;
         }
+        return true;
       });
 }
 
