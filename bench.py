@@ -533,6 +533,8 @@ def run_fqa(args, rank: int, world: int):
     if st != fqa.FQA_OK:
         raise RuntimeError(f"device status {flags:#x} after the corrected steps")
 
+    ulysses = run_ulysses(w0, scale, dev, rank, world, K, ms_per_step) if world > 1 else None
+
     if rank != 0:
         return
     pk, pk_kind = peaks()
@@ -544,7 +546,55 @@ def run_fqa(args, rank: int, world: int):
     cpu = None if args.no_cpu_baseline else cpu_baseline(w, g)
     line = step_line(w, world, K, args.warmup, ms_per_step, attn_ms, quant_ms, bf16_ms, e2e_ms, h2d, d2h,
                      clk.summary(), probe, cpu, traffic_per_launch(), pk, pk_kind, corrected, accuracy)
+    if ulysses is not None:
+        line["ulysses"] = ulysses
     print(json.dumps(line), flush=True)
+
+
+def run_ulysses(w0, scale, dev, rank: int, world: int, K: int, dp_ms: float):
+    """The pages' multi-GPU form ("FLUX 3 Image Klein Base", sections "결과" and
+    "고를 때 기준": Ulysses sequence parallel): one workload's sequence split
+    over the world, all-to-all to head shards, FP8 attention per rank,
+    all-to-all back.  Every rank holds a shard of the same inputs (rank 0's
+    seed); timed like the step (events, barriers, max over ranks)."""
+    import torch
+    import torch.distributed as dist
+
+    from quantized_fp8_attention_b200 import ulysses as uly
+
+    B, H, N, d = w0.B, w0.H, w0.N, w0.d
+    if H % world or N % world or (N // world) % 64:
+        return {"skipped": f"{H} heads / {N} tokens do not split over {world} ranks"}
+    try:
+        g, _ = host_inputs(w0, 0)
+        Nl = N // world
+
+        def shard(bits):
+            x = np.ascontiguousarray(bits[:, :, rank * Nl:(rank + 1) * Nl])
+            return torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
+
+        qs, ks, vs = (shard(g[t]) for t in "qkv")
+        for _ in range(3):
+            uly.ulysses_fp8_attention(qs, ks, vs, scale)
+        torch.cuda.synchronize()
+        Ku = max(4, K // 8)
+        stream = torch.cuda.current_stream()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        dist.barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(Ku):
+            uly.ulysses_fp8_attention(qs, ks, vs, scale)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        dist.barrier()
+        ms = max_over_ranks(e0.elapsed_time(e1) / Ku, dev, world)
+        return {"degree": world, "workload": w0.name, "steps": Ku, "ms_per_step": ms,
+                "tflops": w0.flops / (ms * 1e-3) / 1e12, "scaling": "strong",
+                "step": "all-to-all (q, k, v) + fqa_quantize_a2a + fqa_attention_fp8_a2a + all-to-all (out)",
+                "speedup_vs_one_gpu_step": dp_ms / ms}
+    except Exception as e:  # noqa: BLE001 -- reported in the line, the step's numbers stand
+        return {"error": f"{type(e).__name__}: {e}"}
 
 
 def main():

@@ -65,6 +65,7 @@ struct AttnParams {
   const uint32_t* kmask = nullptr;   // FP8, key-masked kernel: excluded keys [B,H,ceil(N/32)]
   float2* row_stats = nullptr;       // FP8, key-masked kernel: (m, l) per row [B,H,N]
   int out_P = 1;                     // FP8: > 1 writes out in the sequence all-to-all layout
+  int patch = 0;                     // FP8 with kmask: apply it by patching K / V tiles (see attention_fp8.cuh)
 };
 
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {

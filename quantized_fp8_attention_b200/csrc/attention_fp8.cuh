@@ -44,6 +44,15 @@
 // maximum is unchanged), whose V rows stay zero (no term in O).  Their p
 // terms in the row sum are subtracted in the epilogue, from key N-1's score
 // recomputed from its codes.  The softmax loop itself carries no masking.
+// Keys left out by a key mask (the keys an error-corrected pass handles
+// exactly) are either masked in TMEM before the softmax reads a tile
+// (kMaskable), or, when every 64-key block keeps at least one key, patched
+// by the producers (kPatch): each left-out key's K row becomes a copy of the
+// first kept key of its block (same codes and block scale, so the same score:
+// the row maximum is unchanged) and its V row becomes zero (no term in O).
+// The copies' terms stay in the row sum the kernel reports (row_stats); the
+// caller takes them out (the error-corrected merge recomputes the kept keys'
+// scores from the same codes), so the softmax loop is the unmasked one.
 #pragma once
 
 #include "attention.cuh"
@@ -68,8 +77,8 @@ struct F8Traits {
   static constexpr int kOffL = kOffP + 4 * kTileBytes;          // [item parity][tile][half][row]
   static constexpr int kOffBar = kOffL + 2 * 2 * 2 * 128 * 4;
   // fullK, fullV, emptyK, emptyV [kStages]; barQ, barQfree; barS, barSfree,
-  // barP, barPV, barDrain, barL [2 each]; barPatch
-  static constexpr int kNumBars = 4 * kStages + 2 + 12 + 1;
+  // barP, barPV, barDrain, barL [2 each]; barPatch, barPatchV
+  static constexpr int kNumBars = 4 * kStages + 2 + 12 + 2;
   static constexpr int kSmemBytes = kOffBar + 8 * kNumBars + 16 + 1024;
 };
 
@@ -139,7 +148,11 @@ __device__ __forceinline__ void mask_absent_scores(uint32_t tS, uint32_t pw0, ui
 // without it.
 // kShortTail: N is not a multiple of 128 (the patched short last tile above);
 // aligned calls use kShortTail = false and carry none of that code.
-template <bool kShortTail, bool kMaskable>
+// kPatch: the key mask p.kmask applied by patching K and V tiles (above);
+// requires N % 128 == 0 and a kept key in every 64-key block, and writes the
+// row statistics like kMaskable, with l still holding the copies' terms, and
+// leaves O unnormalized (O * sv_max / 448, no division by l).
+template <bool kShortTail, bool kMaskable, bool kPatch = false>
 __global__ void __launch_bounds__(kF8Threads, 1)
     attn_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
@@ -164,7 +177,8 @@ __global__ void __launch_bounds__(kF8Threads, 1)
   uint64_t* barPV = barQ + 8;      // [2] PV_t complete
   uint64_t* barDrain = barQ + 10;  // [2] error path: an issuer's MMAs completed
   uint64_t* barL = barQ + 12;      // [2] both halves' row sums written
-  uint64_t* barPatch = barQ + 14;  // the short last K tile landed (before its patch)
+  uint64_t* barPatch = barQ + 14;  // a K tile to patch landed (before its patch)
+  uint64_t* barPatchV = barQ + 15; // a V tile to patch landed
   float* sL = reinterpret_cast<float*>(smem + T::kOffL);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + T::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -189,6 +203,7 @@ __global__ void __launch_bounds__(kF8Threads, 1)
     mbar_init(barQ, 1);
     mbar_init(barQfree, 2);
     mbar_init(barPatch, 1);
+    mbar_init(barPatchV, 1);
     mbar_init(&barDrain[0], 1);
     mbar_init(&barDrain[1], 1);
     for (int t = 0; t < 2; ++t) {
@@ -235,11 +250,64 @@ __global__ void __launch_bounds__(kF8Threads, 1)
           tma_load_3d(sQ, &tmQ, barQ, 0, w.qp * 2 * kBlockM, head);
           tma_load_3d(sQ + T::kTileBytes, &tmQ, barQ, 0, w.qp * 2 * kBlockM + kBlockM, head);
         }
+        // kPatch: the key-mask words of tile j (left-out keys), loaded a tile
+        // ahead so that their latency overlaps the waits and copies
+        uint32_t kwn[4] = {0u, 0u, 0u, 0u};
+        if constexpr (kPatch) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) kwn[q] = __ldg(p.kmask + (size_t)head * (N / 32) + q);
+        }
         for (int j = 0; j < nkv; ++j, ++g) {
           const int s = g % T::kStages, r = g / T::kStages;
+          uint32_t kw[4] = {kwn[0], kwn[1], kwn[2], kwn[3]};
+          if constexpr (kPatch) {
+            if (j + 1 < nkv) {
+#pragma unroll
+              for (int q = 0; q < 4; ++q) kwn[q] = __ldg(p.kmask + (size_t)head * (N / 32) + 4 * (j + 1) + q);
+            }
+          }
           if (!(ok = mbar_wait(&empty[s], (r & 1) ^ 1, abort_flag, p.status))) break;
           uint8_t* dst = ring + s * T::kTileBytes;
-          if (kShortTail && is_k && j == nkv - 1) {
+          if (kPatch && (kw[0] | kw[1] | kw[2] | kw[3]) != 0u) {
+            // land the tile, then patch the left-out keys' rows: K rows take
+            // the codes of the first kept key of their 64-key block, V rows
+            // become zero; rows are 128 B with 16-byte chunk c of row x at
+            // c ^ (x % 8)
+            uint64_t* pbar = is_k ? barPatch : barPatchV;
+            mbar_arrive_expect_tx(pbar, T::kTileBytes);
+            tma_load_3d(dst, tm, pbar, 0, j * kBlockN, head);
+            if (!(ok = mbar_wait(pbar, patch_phase, abort_flag, p.status))) {
+              mbar_wait_drain(pbar, patch_phase);
+              break;
+            }
+            patch_phase ^= 1u;
+            for (int hb = 0; hb < 2; ++hb) {
+              uint64_t left = ((uint64_t)kw[2 * hb + 1] << 32) | kw[2 * hb];
+              if (left == 0) continue;
+              // (a block with every key left out is excluded by the caller;
+              // the index stays inside the tile regardless)
+              const int f = __ffsll((long long)~left);
+              const int src = 64 * hb + (f > 0 ? f - 1 : 0);
+              uint4 row[8];
+              if (is_k) {
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                  row[c] = *reinterpret_cast<const uint4*>(dst + src * 128 + ((c ^ (src & 7)) << 4));
+              } else {
+#pragma unroll
+                for (int c = 0; c < 8; ++c) row[c] = make_uint4(0u, 0u, 0u, 0u);
+              }
+              while (left != 0) {
+                const int x = 64 * hb + __ffsll((long long)left) - 1;
+                left &= left - 1;
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                  *reinterpret_cast<uint4*>(dst + x * 128 + ((c ^ (x & 7)) << 4)) = row[c];
+              }
+            }
+            fence_proxy_async_smem();            // generic writes -> the MMA's reads
+            mbar_arrive(&full[s]);
+          } else if (kShortTail && is_k && j == nkv - 1) {
             // the short last K tile: land it, then copy key N-1 (tile row
             // valid_last - 1) over the zero-filled rows past N, and only then
             // release it to the MMA.  Rows are 128 B with 16-byte chunk c of
@@ -542,9 +610,11 @@ __global__ void __launch_bounds__(kF8Threads, 1)
       tc_fence_after();
       const bool store = qrow < N;
       // l_row = 0 only when a key mask excluded every key of the row
-      const float fin = (kMaskable && !(l_row > 0.0f)) ? 0.0f : (svmax / 448.0f) / l_row;
+      // (kPatch: O leaves unnormalized, since l still holds the copies' terms)
+      const float fin = kPatch ? svmax / 448.0f
+                               : ((kMaskable && !(l_row > 0.0f)) ? 0.0f : (svmax / 448.0f) / l_row);
       const size_t orow = head * N + (size_t)qrow;
-      if constexpr (kMaskable) {
+      if constexpr (kMaskable || kPatch) {
         if (p.row_stats != nullptr && hf == 0 && store) p.row_stats[orow] = make_float2(m, l_row);
       }
       // the output row: [B,H,N,128], or with out_P > 1 the sequence all-to-all

@@ -130,22 +130,168 @@ __global__ void __launch_bounds__(kSelThreads, 1)
   }
 }
 
+// ------------------------------------------------- patched FP8 part's row sums
+
+// When the FP8 part ran with patched tiles (attn_fp8_kernel<.., kPatch>: each
+// corrected key's K row a copy of the first kept key of its 64-key block, its
+// V row zero), its reported row sum l holds one extra term 2^(x_src - m) per
+// corrected key, x_src the copied key's score.  dup_sum_kernel takes them out:
+// one CTA per (128-row Q tile, head) scores the tile's rows against the copied
+// keys with the same FP8 MMA on the same codes (so the same S), forms x and p
+// exactly as the FP8 softmax does, and writes l - sum_J cnt_J p(src_J) back
+// into the row statistics.  Needs N % 128 == 0 and fewer than 64 corrected
+// keys per head (a kept key in every block; at most 63 copied keys).
+constexpr int kDupThreads = 160;     // warps 0-3: one row each thread; warp 4: lists, TMA, MMA
+constexpr int kDupSmem = 28 * 1024;  // Q8 16 KB + source rows 8 KB; eight CTAs per SM (8 x 64 TMEM columns)
+
+struct DupParams {
+  const uint8_t* k8;        // E4M3 codes [B,H,N,128]
+  const float* sq;          // [B,H,N/64]
+  const float* sk;
+  const uint32_t* kmask;    // [B,H,N/32] corrected keys
+  float2* stats;            // (m, l) per row [B,H,N], l corrected in place
+  int N;
+  float softmax_scale;
+  uint32_t* status;
+};
+
+__global__ void __launch_bounds__(kDupThreads)
+    dup_sum_kernel(const __grid_constant__ CUtensorMap tmQ8, const DupParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sQ8 = smem;                         // 128 rows x 128 B, 128-byte swizzle
+  uint8_t* sKs = smem + 16384;                 // 64 rows x 128 B, 128-byte swizzle
+  __shared__ uint64_t barQ, barS;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+  __shared__ int s_src[64], s_cnt[64], s_blk[64], s_n;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tq = blockIdx.x, head = blockIdx.y, N = p.N, nblk = N / 64;
+  const size_t hbase = (size_t)head * N;
+  if (threadIdx.x == 0) {
+    mbar_init(&barQ, 1);
+    mbar_init(&barS, 1);
+    abort_flag = 0;
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (warp == 4) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&barQ, 16384);
+      tma_load_3d(sQ8, &tmQ8, &barQ, 0, tq * 128, head);
+    }
+    __syncwarp();
+    tmem_alloc(&tmem_slot, 64);
+    tmem_relinquish();
+    // blocks with corrected keys, ascending: the key they copy and their count
+    int n = 0;
+    for (int b0 = 0; b0 < nblk; b0 += 32) {
+      const int J = b0 + lane;
+      int cnt = 0, src = 0;
+      if (J < nblk) {
+        const uint32_t w0 = __ldg(p.kmask + hbase / 32 + 2 * J), w1 = __ldg(p.kmask + hbase / 32 + 2 * J + 1);
+        cnt = __popc(w0) + __popc(w1);
+        const int f = __ffsll((long long)~(((uint64_t)w1 << 32) | w0));
+        src = 64 * J + (f > 0 ? f - 1 : 0);
+      }
+      const uint32_t any = __ballot_sync(0xffffffffu, cnt > 0);
+      const int pos = n + __popc(any & ((1u << lane) - 1u));
+      if (cnt > 0 && pos < 64) {
+        s_src[pos] = src;
+        s_cnt[pos] = cnt;
+        s_blk[pos] = J;
+      }
+      n += __popc(any);
+    }
+    if (lane == 0) s_n = n < 64 ? n : 64;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+  const int nsrc = s_n;
+  // the copied keys' code rows (zero rows past nsrc)
+  for (int w = threadIdx.x; w < 64 * 8; w += kDupThreads) {
+    const int x = w >> 3, c = w & 7;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (x < nsrc) v = __ldg(reinterpret_cast<const uint4*>(p.k8 + (hbase + (size_t)s_src[x]) * 128) + c);
+    *reinterpret_cast<uint4*>(sKs + x * 128 + ((c ^ (x & 7)) << 4)) = v;
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  __syncthreads();
+  if (warp == 4) {
+    if (lane == 0) {
+      if (mbar_wait(&barQ, 0, &abort_flag, p.status)) {
+        tc_fence_after();
+        const uint64_t dQ = make_sdesc_sw128(smem_u32(sQ8), 16, 1024);
+        const uint64_t dK = make_sdesc_sw128(smem_u32(sKs), 16, 1024);
+        constexpr uint32_t kIdesc = make_idesc(0, 0, 128, 64, 0);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) mma_f8_ss(tmem, dQ + 2 * k, dK + 2 * k, kIdesc, k > 0);
+      }
+      tc_commit(&barS);
+    }
+    __syncwarp();
+  } else {
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(&barS, 0, &abort_flag, p.status));
+    tc_fence_after();
+    uint32_t u0[32], u1[32];
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    tmem_ld32(tmem + lane_off, u0);
+    tmem_ld32(tmem + lane_off + 32u, u1);
+    tmem_wait_ld();
+    const int r = threadIdx.x;
+    const size_t row = hbase + (size_t)tq * 128 + r;
+    if (ok && !abort_flag) {
+      const float2 st = p.stats[row];
+      const float c_log2e = p.softmax_scale * 1.4426950408889634f;
+      const float a_row = __ldg(p.sq + (size_t)head * nblk + (tq * 128 + r) / 64);
+      const float nm = -st.x;
+      float dup = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        if (i < nsrc) {
+          // x and p as the FP8 softmax forms them: x = S * a rounded toward
+          // zero, p = 2^(x - m)
+          const float a = a_row * (__ldg(p.sk + (size_t)head * nblk + s_blk[i]) * c_log2e);
+          const float x = __fmul_rz(__uint_as_float(i < 32 ? u0[i] : u1[i - 32]), a);
+          dup = __fmaf_rn((float)s_cnt[i], ex2_approx(__fmaf_rn(x, 1.0f, nm)), dup);
+        }
+      }
+      p.stats[row] = make_float2(st.x, st.y - dup);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 64);
+  }
+}
+
 // ------------------------------------------------------- exact part + merge
 
 constexpr int kCorrThreads = 160;    // warps 0-3: one row each thread; warp 4: TMA, TMEM, MMA
 constexpr int kCorrIssuer = 4;
 
+// kKeys: corrected keys per chunk (128, or 64 when kc <= 64: half the shared
+// memory, so two CTAs share an SM).
+template <int kKeys>
 struct CorrTraits {
-  static constexpr int kTileBytes = 128 * 128 * 2;                // BF16, two 64-column halves
+  static constexpr int kQBytes = 128 * 128 * 2;                   // BF16 Q tile, two 64-channel halves
+  static constexpr int kKVHalf = kKeys * 128;                     // one 64-channel half of K_c or V_c
+  static constexpr int kPBytes = 128 * kKeys * 2;                 // P (hi or lo): 64-key halves of 16 KB
   static constexpr int kOffQ = 0;
-  static constexpr int kOffK = kOffQ + kTileBytes;
-  static constexpr int kOffV = kOffK + kTileBytes;
-  static constexpr int kOffPhi = kOffV + kTileBytes;
-  static constexpr int kOffPlo = kOffPhi + kTileBytes;
-  static constexpr int kOffBar = kOffPlo + kTileBytes;
+  static constexpr int kOffK = kOffQ + kQBytes;
+  static constexpr int kOffV = kOffK + 2 * kKVHalf;
+  static constexpr int kOffPhi = kOffV + 2 * kKVHalf;
+  static constexpr int kOffPlo = kOffPhi + kPBytes;
+  static constexpr int kOffBar = kOffPlo + kPBytes;
   static constexpr int kNumBars = 4;                               // barQ, barS, barP, barPV
   static constexpr int kSmemBytes = kOffBar + 8 * kNumBars + 16 + 1024;
-  static constexpr uint32_t kIdescS = make_idesc(1, 1, 128, 128, 0);
+  static constexpr int kCtasPerSm = kKeys == 64 ? 2 : 1;
+  static constexpr uint32_t kIdescS = make_idesc(1, 1, 128, kKeys, 0);
   static constexpr uint32_t kIdescPV = make_idesc(1, 1, 128, 128, 1);
 };
 
@@ -155,8 +301,9 @@ struct CorrParams {
   const __nv_bfloat16* v;
   const float* k_mean;      // [B,H,128]
   const int* idx;           // [B,H,kc] corrected keys, ascending
-  const float* o1;          // FP8 part's FP32 output [B,H,N,128] (normalized)
+  const float* o1;          // FP8 part's FP32 output [B,H,N,128]: normalized by l1, or not (o1_raw)
   const float2* stats;      // FP8 part's (m1, l1) per row [B,H,N]
+  int o1_raw;               // o1 is unnormalized (the patched FP8 part)
   void* out;                // [B,H,N,128] BF16 or FP32
   int out_f32;
   int B, H, N, kc;
@@ -164,15 +311,17 @@ struct CorrParams {
   uint32_t* status;
 };
 
-// 16-byte chunk c (8 BF16 values) of row x of a 128-row operand tile: two
-// 64-column halves of 16 KB, 128 B per row, chunk c of a half at c ^ (x % 8).
-__device__ __forceinline__ uint32_t tile_chunk_off(int x, int c) {
-  return (uint32_t)((c >> 3) * 16384 + x * 128 + (((c & 7) ^ (x & 7)) << 4));
+// 16-byte chunk c (8 BF16 values) of row x of an operand tile stored as two
+// 64-column halves `half` bytes apart, 128 B per row, chunk c of a half at
+// c ^ (x % 8) (128-byte swizzle).
+__device__ __forceinline__ uint32_t tile_chunk_off(int x, int c, int half) {
+  return (uint32_t)((c >> 3) * half + x * 128 + (((c & 7) ^ (x & 7)) << 4));
 }
 
-__global__ void __launch_bounds__(kCorrThreads, 1)
+template <int kKeys>
+__global__ void __launch_bounds__(kCorrThreads, CorrTraits<kKeys>::kCtasPerSm)
     correct_kernel(const __grid_constant__ CUtensorMap tmQ, const CorrParams p) {
-  using T = CorrTraits;
+  using T = CorrTraits<kKeys>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -191,7 +340,10 @@ __global__ void __launch_bounds__(kCorrThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int head = blockIdx.y, N = p.N, kc = p.kc;
-  const int ntq = (N + 127) / 128, nch = (kc + 127) / 128;
+  const int ntq = (N + 127) / 128, nch = (kc + kKeys - 1) / kKeys;
+  // 64-key instance: q . mu from the S MMA (K_c rows 61..63 hold mu), so
+  // kc <= 61 there; the 128-key one sums q . mu per row thread
+  constexpr bool kMuRows = kKeys == 64;
   const float c_log2e = p.softmax_scale * 1.4426950408889634f;
   const size_t hbase = (size_t)head * N;
 
@@ -204,7 +356,7 @@ __global__ void __launch_bounds__(kCorrThreads, 1)
     mbar_fence_init();
   }
   if (warp == kCorrIssuer) {
-    tmem_alloc(tmem_slot, 256);               // S [0,128), O [128,256)
+    tmem_alloc(tmem_slot, 256);               // S [0,kKeys), O [128,256)
     tmem_relinquish();
   }
   tc_fence_before();
@@ -212,40 +364,63 @@ __global__ void __launch_bounds__(kCorrThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  // corrected keys [128 ch, 128 ch + 128) of this head -> sK, sV (zero rows
-  // past kc), all threads; made visible to the tensor core
+  // corrected keys [kKeys ch, kKeys ch + kKeys) of this head -> sK, sV (zero
+  // rows past kc), all threads; made visible to the tensor core
   auto gather = [&](int ch) {
-    const int* ids = p.idx + (size_t)head * kc + 128 * ch;
-    const int nk = min(128, kc - 128 * ch);
-    for (int w = threadIdx.x; w < 128 * 16; w += kCorrThreads) {
+    const int* ids = p.idx + (size_t)head * kc + kKeys * ch;
+    const int nk = min(kKeys, kc - kKeys * ch);
+    for (int w = threadIdx.x; w < kKeys * 16; w += kCorrThreads) {
       const int x = w >> 4, c = w & 15;
       uint4 kv = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
       if (x < nk) {
         const size_t row = hbase + (size_t)__ldg(ids + x);
         kv = __ldg(reinterpret_cast<const uint4*>(p.k + row * 128) + c);
         vv = __ldg(reinterpret_cast<const uint4*>(p.v + row * 128) + c);
+      } else if (kMuRows && x >= kKeys - 3) {
+        // mu = hi + mid + lo in BF16 (mu - hi - mid - lo is below 2^-24 |mu|),
+        // so that the S MMA also gives q . mu in its last three columns
+        const int part = x - (kKeys - 3);
+        const float* mu = p.k_mean + (size_t)head * 128 + 8 * c;
+        uint32_t wv[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float pr[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const float m0 = __ldg(mu + 2 * e + h);
+            const float hi = __bfloat162float(__float2bfloat16_rn(m0));
+            const float mid = __bfloat162float(__float2bfloat16_rn(m0 - hi));
+            const float lo = __bfloat162float(__float2bfloat16_rn((m0 - hi) - mid));
+            pr[h] = part == 0 ? hi : (part == 1 ? mid : lo);
+          }
+          const __nv_bfloat162 b2 = __floats2bfloat162_rn(pr[0], pr[1]);
+          wv[e] = *reinterpret_cast<const uint32_t*>(&b2);
+        }
+        kv = make_uint4(wv[0], wv[1], wv[2], wv[3]);
       }
-      *reinterpret_cast<uint4*>(sK + tile_chunk_off(x, c)) = kv;
-      *reinterpret_cast<uint4*>(sV + tile_chunk_off(x, c)) = vv;
+      *reinterpret_cast<uint4*>(sK + tile_chunk_off(x, c, T::kKVHalf)) = kv;
+      *reinterpret_cast<uint4*>(sV + tile_chunk_off(x, c, T::kKVHalf)) = vv;
     }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     __syncthreads();
   };
   if (nch == 1) gather(0);
 
+  // the first Q tile; later ones are loaded as soon as the last S MMA of the
+  // tile before has read sQ
+  if (warp == kCorrIssuer && lane == 0 && (int)blockIdx.x < ntq) {
+    mbar_arrive_expect_tx(barQ, T::kQBytes);
+    tma_load_3d(sQ, &tmQ, barQ, 0, (int)blockIdx.x * 128, head);
+    tma_load_3d(sQ + 16384, &tmQ, barQ, 64, (int)blockIdx.x * 128, head);
+  }
   uint32_t ph_q = 0, ph_s = 0, ph_p = 0, ph_pv = 0;
   bool ok = true;
   for (int tq = blockIdx.x; tq < ntq; tq += gridDim.x) {
-    if (warp == kCorrIssuer && lane == 0) {
-      mbar_arrive_expect_tx(barQ, T::kTileBytes);
-      tma_load_3d(sQ, &tmQ, barQ, 0, tq * 128, head);
-      tma_load_3d(sQ + 16384, &tmQ, barQ, 64, tq * 128, head);
-    }
     const int r = threadIdx.x & 127;           // row of the tile (row threads)
     const int qrow = tq * 128 + r;
-    // q . mu for this row, from the BF16 row in global memory
+    // q . mu for this row, from the BF16 row in global memory (128-key instance)
     float qmu = 0.0f;
-    if (warp < 4 && qrow < N) {
+    if (!kMuRows && warp < 4 && qrow < N) {
       const uint4* qr = reinterpret_cast<const uint4*>(p.q + (hbase + qrow) * 128);
       const float* mu = p.k_mean + (size_t)head * 128;
 #pragma unroll 4
@@ -263,7 +438,7 @@ __global__ void __launch_bounds__(kCorrThreads, 1)
     float m2 = -INFINITY, l2 = 0.0f;
     for (int ch = 0; ch < nch; ++ch) {
       if (nch > 1) gather(ch);
-      const int nk = min(128, kc - 128 * ch);
+      const int nk = min(kKeys, kc - kKeys * ch);
       if (warp == kCorrIssuer) {
         if (lane == 0) {
           if (ch == 0) {
@@ -275,11 +450,22 @@ __global__ void __launch_bounds__(kCorrThreads, 1)
             const uint64_t dQ = make_sdesc_sw128(smem_u32(sQ), 16, 1024);
             const uint64_t dK = make_sdesc_sw128(smem_u32(sK), 16, 1024);
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const uint64_t off = (uint64_t)((k >> 2) * 1024 + (k & 3) * 2);
-              mma_bf16_ss(tmem, dQ + off, dK + off, T::kIdescS, k > 0);
+            for (int k = 0; k < 8; ++k) {           // 16 channels per MMA
+              const uint64_t oq = (uint64_t)((k >> 2) * (16384 >> 4) + (k & 3) * 2);
+              const uint64_t ok2 = (uint64_t)((k >> 2) * (T::kKVHalf >> 4) + (k & 3) * 2);
+              mma_bf16_ss(tmem, dQ + oq, dK + ok2, T::kIdescS, k > 0);
             }
             tc_commit(barS);
+            if (ch == nch - 1 && tq + (int)gridDim.x < ntq) {
+              // sQ is free once this S completed: load the next tile's Q
+              if (mbar_wait(barS, ph_s, abort_flag, p.status)) {
+                mbar_arrive_expect_tx(barQ, T::kQBytes);
+                tma_load_3d(sQ, &tmQ, barQ, 0, (tq + (int)gridDim.x) * 128, head);
+                tma_load_3d(sQ + 16384, &tmQ, barQ, 64, (tq + (int)gridDim.x) * 128, head);
+              } else {
+                ok = false;
+              }
+            }
           }
         }
         __syncwarp();
@@ -288,24 +474,24 @@ __global__ void __launch_bounds__(kCorrThreads, 1)
         ok = __all_sync(0xffffffffu, mbar_wait(barS, ph_s, abort_flag, p.status));
         tc_fence_after();
         const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-        float x[128];
+        float x[kKeys];
+        uint32_t u[kKeys];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t u[32];
-          tmem_ld32(tmem + lane_off + 32u * c, u);
-          tmem_wait_ld();
+        for (int c = 0; c < kKeys / 32; ++c) tmem_ld32(tmem + lane_off + 32u * c, *reinterpret_cast<uint32_t(*)[32]>(&u[32 * c]));
+        tmem_wait_ld();
+        if constexpr (kMuRows)
+          qmu = (__uint_as_float(u[kKeys - 3]) + __uint_as_float(u[kKeys - 2])) + __uint_as_float(u[kKeys - 1]);
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            x[32 * c + e] = (32 * c + e < nk) ? (__uint_as_float(u[e]) - qmu) * c_log2e : -INFINITY;
-        }
+        for (int e = 0; e < kKeys; ++e)
+          x[e] = (e < nk) ? (__uint_as_float(u[e]) - qmu) * c_log2e : -INFINITY;
         float tmax = x[0];
 #pragma unroll
-        for (int e = 1; e < 128; ++e) tmax = fmaxf(tmax, x[e]);
+        for (int e = 1; e < kKeys; ++e) tmax = fmaxf(tmax, x[e]);
         const float m_new = fmaxf(m2, tmax);
         const float alpha = m2 == -INFINITY ? 0.0f : ex2_approx(m2 - m_new);
         float ls = 0.0f;
 #pragma unroll
-        for (int c8 = 0; c8 < 16; ++c8) {
+        for (int c8 = 0; c8 < kKeys / 8; ++c8) {
           uint32_t hw[4], lw[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -318,7 +504,7 @@ __global__ void __launch_bounds__(kCorrThreads, 1)
             hw[e] = *reinterpret_cast<const uint32_t*>(&h);
             lw[e] = *reinterpret_cast<const uint32_t*>(&lo);
           }
-          const uint32_t off = tile_chunk_off(r, c8);
+          const uint32_t off = tile_chunk_off(r, c8, 16384);
           *reinterpret_cast<uint4*>(sPhi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
           *reinterpret_cast<uint4*>(sPlo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
         }
@@ -353,10 +539,10 @@ __global__ void __launch_bounds__(kCorrThreads, 1)
             tc_fence_after();
             const uint64_t dPh = make_sdesc_sw128(smem_u32(sPhi), 16, 1024);
             const uint64_t dPl = make_sdesc_sw128(smem_u32(sPlo), 16, 1024);
-            const uint64_t dV = make_sdesc_sw128(smem_u32(sV), 16384, 1024);
+            const uint64_t dV = make_sdesc_sw128(smem_u32(sV), T::kKVHalf, 1024);
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const uint64_t offp = (uint64_t)((k >> 2) * 1024 + (k & 3) * 2);
+            for (int k = 0; k < kKeys / 16; ++k) {  // 16 keys per MMA
+              const uint64_t offp = (uint64_t)((k >> 2) * (16384 >> 4) + (k & 3) * 2);
               mma_bf16_ss(tmem + 128u, dPh + offp, dV + 128u * k, T::kIdescPV, ch > 0 || k > 0);
               mma_bf16_ss(tmem + 128u, dPl + offp, dV + 128u * k, T::kIdescPV, 1);
             }
@@ -390,40 +576,50 @@ __global__ void __launch_bounds__(kCorrThreads, 1)
         const float L = l1 * w1 + l2 * w2;
         inv = L > 0.0f ? 1.0f / L : 0.0f;
       }
-      const float a1 = l1 * w1 * inv, a2 = w2 * inv;
+      const float a1 = (p.o1_raw ? w1 : l1 * w1) * inv, a2 = w2 * inv;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t o[32];
-        tmem_ld32(tmem + 128u + lane_off + 32u * c, o);
-        tmem_wait_ld();
-        if (!store) continue;
-        float res[32];
-        const float4* s1 = reinterpret_cast<const float4*>(o1r + 32 * c);
+      for (int c2 = 0; c2 < 4; c2 += 2) {
+        // two 32-column chunks per round trip: both halves' O1 loads in flight
+        float4 f1[16];
+        if (store) {
+          const float4* s1 = reinterpret_cast<const float4*>(o1r + 32 * c2);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float4 f = __ldg(s1 + e);
-          res[4 * e] = f.x * a1 + __uint_as_float(o[4 * e]) * a2;
-          res[4 * e + 1] = f.y * a1 + __uint_as_float(o[4 * e + 1]) * a2;
-          res[4 * e + 2] = f.z * a1 + __uint_as_float(o[4 * e + 2]) * a2;
-          res[4 * e + 3] = f.w * a1 + __uint_as_float(o[4 * e + 3]) * a2;
+          for (int e = 0; e < 16; ++e) f1[e] = __ldg(s1 + e);
         }
-        const size_t orow = hbase + qrow;
-        if (p.out_f32) {
-          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow * 128 + 32 * c);
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            dst[e] = make_float4(res[4 * e], res[4 * e + 1], res[4 * e + 2], res[4 * e + 3]);
-        } else {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + orow * 128 + 32 * c);
+        for (int h = 0; h < 2; ++h) {
+          const int c = c2 + h;
+          uint32_t o[32];
+          tmem_ld32(tmem + 128u + lane_off + 32u * c, o);
+          tmem_wait_ld();
+          if (!store) continue;
+          float res[32];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            uint32_t w4[4];
+          for (int e = 0; e < 8; ++e) {
+            const float4 f = f1[8 * h + e];
+            res[4 * e] = f.x * a1 + __uint_as_float(o[4 * e]) * a2;
+            res[4 * e + 1] = f.y * a1 + __uint_as_float(o[4 * e + 1]) * a2;
+            res[4 * e + 2] = f.z * a1 + __uint_as_float(o[4 * e + 2]) * a2;
+            res[4 * e + 3] = f.w * a1 + __uint_as_float(o[4 * e + 3]) * a2;
+          }
+          const size_t orow = hbase + qrow;
+          if (p.out_f32) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow * 128 + 32 * c);
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const __nv_bfloat162 b2 = __floats2bfloat162_rn(res[8 * e + 2 * u], res[8 * e + 2 * u + 1]);
-              w4[u] = *reinterpret_cast<const uint32_t*>(&b2);
+            for (int e = 0; e < 8; ++e)
+              dst[e] = make_float4(res[4 * e], res[4 * e + 1], res[4 * e + 2], res[4 * e + 3]);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + orow * 128 + 32 * c);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              uint32_t w4[4];
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const __nv_bfloat162 b2 = __floats2bfloat162_rn(res[8 * e + 2 * u], res[8 * e + 2 * u + 1]);
+                w4[u] = *reinterpret_cast<const uint32_t*>(&b2);
+              }
+              dst[e] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
             }
-            dst[e] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
           }
         }
       }

@@ -170,8 +170,11 @@ static fqa_status launch_attention_fp8(const void* q, const void* k, const void*
   const bool tail = prm.N % kBlockN != 0;
   const bool masked = prm.kmask != nullptr || prm.row_stats != nullptr;
   using KernelFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const AttnParams);
-  const KernelFn fn = tail ? (masked ? attn_fp8_kernel<true, true> : attn_fp8_kernel<true, false>)
-                           : (masked ? attn_fp8_kernel<false, true> : attn_fp8_kernel<false, false>);
+  KernelFn fn = tail ? (masked ? attn_fp8_kernel<true, true> : attn_fp8_kernel<true, false>)
+                     : (masked ? attn_fp8_kernel<false, true> : attn_fp8_kernel<false, false>);
+  // a key mask that leaves a key in every 64-key block of an aligned N:
+  // patched tiles instead of masking (the caller checks the condition)
+  if (prm.patch && !tail && prm.kmask != nullptr) fn = attn_fp8_kernel<false, false, true>;
   if (cudaFuncSetAttribute((const void*)fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            F8Traits::kSmemBytes) != cudaSuccess)
     return FQA_ERR_CUDA;
@@ -465,22 +468,42 @@ fqa_status fqa_attention_fp8_corrected(const void* q, const void* k, const void*
   prm.k8 = static_cast<const uint8_t*>(k8);
   prm.kmask = kmask;
   prm.row_stats = stats;
+  // fewer than 64 corrected keys per head leave a kept key in every 64-key
+  // block: the key mask can be applied by patching tiles
+  prm.patch = (kc < 64 && N % kBlockN == 0) ? 1 : 0;
   if ((st = launch_attention_fp8(q8, k8, v8, prm, s)) != FQA_OK) return st;
-  // exact part over the corrected keys, merged into the output
+  if (prm.patch) {
+    // take the copied keys' terms out of the patched FP8 part's row sums
+    CUtensorMap tq8;
+    if (!make_tmap(&tq8, q8, true, N, B * H)) return FQA_ERR_CUDA;
+    if (cudaFuncSetAttribute(dup_sum_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDupSmem) !=
+        cudaSuccess)
+      return FQA_ERR_CUDA;
+    DupParams dp{static_cast<const uint8_t*>(k8), sq, sk, kmask, stats, N, softmax_scale, status};
+    dup_sum_kernel<<<dim3(N / kBlockM, B * H), kDupThreads, kDupSmem, s>>>(tq8, dp);
+    if ((st = launch_status()) != FQA_OK) return st;
+  }
+  // exact part over the corrected keys, merged into the output: one chunk of
+  // 64 (two CTAs per SM; three of its rows carry the K mean) when they fit
   CUtensorMap tq;
   if (!make_tmap(&tq, q, false, N, B * H)) return FQA_ERR_CUDA;
-  if (cudaFuncSetAttribute(correct_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           CorrTraits::kSmemBytes) != cudaSuccess)
-    return FQA_ERR_CUDA;
   CorrParams cp{static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-                static_cast<const __nv_bfloat16*>(v), k_mean, idx, o1, stats, out,
+                static_cast<const __nv_bfloat16*>(v), k_mean, idx, o1, stats, prm.patch, out,
                 out_dtype == FQA_OUT_F32, B, H, N, kc, softmax_scale, status};
-  const int sms = num_sms();
+  const bool small = kc <= 61;
+  const void* fn = small ? (const void*)correct_kernel<64> : (const void*)correct_kernel<128>;
+  const int smem = small ? CorrTraits<64>::kSmemBytes : CorrTraits<128>::kSmemBytes;
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return FQA_ERR_CUDA;
+  const int sms = num_sms() * (small ? CorrTraits<64>::kCtasPerSm : CorrTraits<128>::kCtasPerSm);
   const int ntq = (N + 127) / 128;
   int split = (sms + B * H - 1) / (B * H);       // about one wave of CTAs
   if (split > ntq) split = ntq;
   if (split < 1) split = 1;
-  correct_kernel<<<dim3(split, B * H), kCorrThreads, CorrTraits::kSmemBytes, s>>>(tq, cp);
+  if (small)
+    correct_kernel<64><<<dim3(split, B * H), kCorrThreads, smem, s>>>(tq, cp);
+  else
+    correct_kernel<128><<<dim3(split, B * H), kCorrThreads, smem, s>>>(tq, cp);
   return launch_status();
 }
 
