@@ -223,6 +223,15 @@ def run_sweep(args):
         cws = fqa.alloc_corrected_workspace(w.B, w.H, w.N, 0.005, dev)
         ms_c = timed(lambda: fqa.attention_fp8_corrected(q, k, v, qz, k_err, scale, 0.005, fqa.FQA_OUT_BF16,
                                                          out=out, workspace=cws), reps(1000))
+        # NVFP4 Q.K (N a multiple of 128): the FP4 quantizer and the attention
+        nv = None
+        if w.N % 128 == 0:
+            fqa.quantize(q, k, v, out=qz, workspace=ws)
+            qn = fqa.quantize_nvfp4_qk(q, k, qz.k_mean)
+            ms_n = timed(lambda: fqa.attention_nvfp4(qn, qz, scale, fqa.FQA_OUT_BF16, out=out), reps(650))
+            ms_nq = timed(lambda: fqa.quantize_nvfp4_qk(q, k, qz.k_mean, out=qn), 100, pre=lambda: flush.fill_(1))
+            nv = {"ms": ms_n, "tflops": w.flops / ms_n / 1e9, "time_vs_fp8": ms_n / ms_a,
+                  "quantize_nvfp4_qk_ms": ms_nq}
         st, flags = fqa.fqa_debug_status()
         if st != fqa.FQA_OK:
             raise RuntimeError(f"device status {flags:#x} on {w.name}")
@@ -236,6 +245,7 @@ def run_sweep(args):
                                         "time_vs_fp8": ms_c / ms_a, "time_vs_bf16": ms_c / ms_b},
             "attention_bf16": {"ms": ms_b, "tflops": w.flops / ms_b / 1e9,
                                "frac_of_bf16_peak": w.flops / ms_b / 1e9 / pk["bf16_tflops"]},
+            "attention_nvfp4": nv,
             "quantizer": {"ms": ms_q, "gbs": qbytes / ms_q / 1e6, "frac_of_hbm": qbytes / ms_q / 1e6 / pk["hbm_gbs"],
                           "l2": "flushed before every launch"},
             "peaks": pk_kind}), flush=True)
@@ -314,11 +324,15 @@ def accuracy_sample(w, g, q, k, v, scale, rho, qz, k_err, out, cws):
     plain = cos(fqa.attention_fp8(qz, scale, fqa.FQA_OUT_F32))
     fqa.quantize_keyerr(q, k, v, out=qz, k_err=k_err)
     corr = cos(fqa.attention_fp8_corrected(q, k, v, qz, k_err, scale, rho, fqa.FQA_OUT_F32, workspace=cws))
+    nv = None
+    if w.N % 128 == 0:
+        fqa.quantize(q, k, v, out=qz)
+        nv = cos(fqa.attention_nvfp4(fqa.quantize_nvfp4_qk(q, k, qz.k_mean), qz, scale, fqa.FQA_OUT_F32))
     sample = f"heads {heads}, rows [0,128) u [N/2, N/2+128) u [N-128, N), all keys"
     accuracy = {"cos_vs_exact_fp64": plain, "target": 0.995, "meets_target": plain >= 0.995, "sample": sample}
     corrected = {"rho": rho, "keys_per_head": fqa.fqa_corrected_keys(w.N, rho), "cos_vs_exact_fp64": corr,
                  "meets_target": corr >= 0.995}
-    return accuracy, corrected
+    return accuracy, corrected, nv
 
 
 # ------------------------------------------------------------ CPU baseline
@@ -533,13 +547,37 @@ def run_fqa(args, rank: int, world: int):
     if st != fqa.FQA_OK:
         raise RuntimeError(f"device status {flags:#x} after the corrected steps")
 
+    # NVFP4 Q.K with FP8 P.V, same inputs: the FP8 quantizer (V codes and the K
+    # mean), the NVFP4 quantizer of Q and smoothed K, the attention
+    nv_ms = None
+    if N % 128 == 0:
+        qn = fqa.alloc_quantized_nvfp4(B, H, N, dev)
+
+        def nvfp4_step():
+            fqa.quantize(q, k, v, out=qz, workspace=ws)
+            fqa.quantize_nvfp4_qk(q, k, qz.k_mean, out=qn)
+            fqa.attention_nvfp4(qn, qz, scale, fqa.FQA_OUT_BF16, out=out)
+
+        for _ in range(3):
+            nvfp4_step()
+        Kn = max(1, K // 4)
+        e0.record(stream)
+        for _ in range(Kn):
+            nvfp4_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        nv_ms = e0.elapsed_time(e1) / Kn
+        st, flags = fqa.fqa_debug_status()
+        if st != fqa.FQA_OK:
+            raise RuntimeError(f"device status {flags:#x} after the NVFP4 steps")
+
     ulysses = run_ulysses(w0, scale, dev, rank, world, K, ms_per_step) if world > 1 else None
 
     if rank != 0:
         return
     pk, pk_kind = peaks()
     probe = fp8_gemm_probe(dev)
-    accuracy, corrected = accuracy_sample(w, g, q, k, v, scale, rho, qz, k_err, out, cws)
+    accuracy, corrected, nv_cos = accuracy_sample(w, g, q, k, v, scale, rho, qz, k_err, out, cws)
     corrected.update({"ms_per_step": corr_ms, "step": "fqa_quantize_keyerr + fqa_attention_fp8_corrected",
                       "tflops": flops / (corr_ms * 1e-3) / 1e12,
                       "time_vs_fp8_step": corr_ms / ms_per_step, "time_vs_bf16_attention": corr_ms / bf16_ms})
@@ -548,6 +586,10 @@ def run_fqa(args, rank: int, world: int):
                      clk.summary(), probe, cpu, traffic_per_launch(), pk, pk_kind, corrected, accuracy)
     if ulysses is not None:
         line["ulysses"] = ulysses
+    if nv_ms is not None:
+        line["nvfp4"] = {"ms_per_step": nv_ms, "tflops": flops / (nv_ms * 1e-3) / 1e12,
+                         "step": "fqa_quantize + fqa_quantize_nvfp4_qk + fqa_attention_nvfp4",
+                         "time_vs_fp8_step": nv_ms / ms_per_step, "cos_vs_exact_fp64": nv_cos}
     print(json.dumps(line), flush=True)
 
 
