@@ -30,23 +30,14 @@ constexpr int kBlockM = 128;   // query rows per CTA
 constexpr int kBlockN = 128;   // keys per KV tile (part of the FP8 rounding rule)
 constexpr int kMaxScaleBlocks = 1024;   // N <= 65536
 
-// Of every 8 exponentials (pairs of keys) this many are evaluated by the FMA
-// pipe polynomial instead of the MUFU ex2 unit, to balance the two pipes.
-#ifndef FQA_EXP2_POLY_PER8
-#define FQA_EXP2_POLY_PER8 0
-#endif
-constexpr int kPolyPer8 = FQA_EXP2_POLY_PER8;
-
 // p for two keys at once: 2^(x - m) with x = fl(S * a) already rounded and
 // m = max x.  x - m is exact near the maximum (Sterbenz), so the row maximum
 // gets p = 1 exactly and the row sum l carries no common rounding factor (a
 // fused S * a - m would give the maximum p = 2^delta, delta the rounding
 // residue of m, and bias l by ~|m| 2^-24).  The subtraction is written as
 // fma(x, 1, -m) so that the multiply producing x can never be fused into it.
-template <bool kPoly>
 __device__ __forceinline__ float2 exp2_pair(float2 x, float2 nm2) {
   const float2 d = f2_fma(x, make_float2(1.0f, 1.0f), nm2);
-  if constexpr (kPoly) return exp2_poly2(d);
   return make_float2(ex2_approx(d.x), ex2_approx(d.y));
 }
 

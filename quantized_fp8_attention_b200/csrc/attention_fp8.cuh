@@ -533,11 +533,8 @@ __global__ void __launch_bounds__(kF8Threads, 1)
             const uint32_t* u = &sr[4 * w4];
             const float2 x01 = f2_mul_rz(make_float2(__uint_as_float(u[0]), __uint_as_float(u[1])), a2);
             const float2 x23 = f2_mul_rz(make_float2(__uint_as_float(u[2]), __uint_as_float(u[3])), a2);
-            const int e = 16 * ch + 2 * w4;
-            // pairs with (index % 8) < kPolyPer8 take the FMA-pipe exp2
-            const float2 p01 = (e % 8) < kPolyPer8 ? exp2_pair<true>(x01, nm2) : exp2_pair<false>(x01, nm2);
-            const float2 p23 = ((e + 1) % 8) < kPolyPer8 ? exp2_pair<true>(x23, nm2)
-                                                         : exp2_pair<false>(x23, nm2);
+            const float2 p01 = exp2_pair(x01, nm2);
+            const float2 p23 = exp2_pair(x23, nm2);
             ls[0] = f2_add(ls[0], p01);
             ls[1] = f2_add(ls[1], p23);
             const float2 q01 = f2_mul(p01, c2), q23 = f2_mul(p23, c2);

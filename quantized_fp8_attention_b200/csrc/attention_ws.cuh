@@ -332,8 +332,7 @@ __global__ void __launch_bounds__(kWsThreads, 1)
 #pragma unroll
             for (int u = 0; u < 16; ++u) {
               const int e = 16 * ch + u;
-              const float2 pp = ((u % 8) < kPolyPer8) ? exp2_pair<true>(X[e], nm2)
-                                                      : exp2_pair<false>(X[e], nm2);
+              const float2 pp = exp2_pair(X[e], nm2);
               ls[u & 1] = f2_add(ls[u & 1], pp);
               __nv_bfloat162 pb = __floats2bfloat162_rn(pp.x, pp.y);
               pw[u] = *reinterpret_cast<uint32_t*>(&pb);

@@ -369,38 +369,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-// 2^x for x <= 0 on the FMA pipe, for two values at once.  Cody-Waite style
-// reduction x = n + f with n = rint(x), f in [-1/2, 1/2] (n from the
-// 1.5 * 2^23 magic-number addition), 2^f from a degree-5 minimax polynomial
-// (Remez exchange on the relative error; coefficients rounded to binary32 by
-// tools/fit_exp2_poly.py: max relative error 1.5e-7 before the binary32
-// Horner roundings), and 2^n by adding n to the exponent field.  Inputs are
-// clamped at -126 so the exponent field cannot wrap; 2^-126 is far below what
-// an E4M3 code or a row sum can resolve.
-constexpr float kExp2C0 = 1.0000001192092896f;     // 0x3f800001
-constexpr float kExp2C1 = 0.6931469440460205f;     // 0x3f317214
-constexpr float kExp2C2 = 0.24022120237350464f;    // 0x3e75fc8c
-constexpr float kExp2C3 = 0.05550713092088699f;    // 0x3d635b72
-constexpr float kExp2C4 = 0.009675540961325169f;   // 0x3c1e8629
-constexpr float kExp2C5 = 0.0013276472454890609f;  // 0x3aae0473
-
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  x.x = fmaxf(x.x, -126.0f);
-  x.y = fmaxf(x.y, -126.0f);
-  const float2 magic = make_float2(12582912.0f, 12582912.0f);   // 1.5 * 2^23
-  const float2 t = f2_add(x, magic);                             // n in the low mantissa bits
-  const float2 n = f2_add(t, make_float2(-12582912.0f, -12582912.0f));
-  const float2 f = f2_add(x, make_float2(-n.x, -n.y));
-  float2 p = f2_fma(make_float2(kExp2C5, kExp2C5), f, make_float2(kExp2C4, kExp2C4));
-  p = f2_fma(p, f, make_float2(kExp2C3, kExp2C3));
-  p = f2_fma(p, f, make_float2(kExp2C2, kExp2C2));
-  p = f2_fma(p, f, make_float2(kExp2C1, kExp2C1));
-  p = f2_fma(p, f, make_float2(kExp2C0, kExp2C0));
-  // (bits(t) << 23) == n << 23 modulo 2^32: the magic number's low 9 bits are 0
-  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
-                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
-}
-
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
