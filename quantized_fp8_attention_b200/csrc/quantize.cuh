@@ -55,12 +55,12 @@ constexpr int kChunks = kBlockBytes / 16 / kQuantThreads;       // 16-byte chunk
 constexpr int kVals = 8 * kChunks;
 constexpr int kRingBytes = 48 * 1024;             // four CTAs per SM
 constexpr int kMaxSlots = kRingBytes / kBlockBytes;
-constexpr int kQuantSmem = kRingBytes + 128;
+constexpr int kSideBytes = kHeadDim * 4;           // per slot: a head's k_mean row (phase 3)
+constexpr int kQuantSmem = kRingBytes + kMaxSlots * kSideBytes + 128;
 constexpr int kPartialRowsPerSlot = kBlockBytes / (kHeadDim * 4);   // 32 partial rows per 16 KB
 // CTAs the shared memory admits per SM (the register cap follows from it)
 constexpr int kQuantMinCtas = (228 * 1024) / (kQuantSmem + 2048) < 1 ? 1 : (228 * 1024) / (kQuantSmem + 2048);
 static_assert(kMaxSlots >= 3 && kMaxSlots <= 32, "ring size");
-static_assert(kRingBytes / (kBlockBytes + kHeadDim * 4) >= 2, "two slots in every pass");
 static_assert(kQuantThreads >= 2 * kHeadDim, "k_mean and sv_max threads");
 static_assert((kQuantThreads * 8) % kHeadDim == 0, "chunk c of thread t starts at channel 8t mod 128");
 
@@ -207,6 +207,7 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantMinCtas) quantize_fused_k
     uint32_t* status, float* __restrict__ k_err, int in_P) {
   extern __shared__ uint8_t qsmem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(qsmem_raw) + 127) & ~uintptr_t(127));
+  uint8_t* side = ring + kRingBytes;               // kMaxSlots x kSideBytes
   __shared__ uint64_t full[kMaxSlots];
   __shared__ int slot_unit[kMaxSlots];
   __shared__ float red[2 * kQuantWarps];
@@ -405,19 +406,20 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantMinCtas) quantize_fused_k
   if (!failed && !pass_qv(q, q8, sq, queue(kCtrQB, nqa, nunits, false))) failed = 1;
   if (!grid_wait(&ctr[kCtrBarrier], 2, status, &failed)) return;
 
-  // ---- phase 3: K codes, newest units of phase 1b first.  Each slot holds
-  // the unit's K block and its head's k_mean row (512 B), loaded together.
-  constexpr int kSlot3 = kBlockBytes + kHeadDim * 4;
-  run(kSlot3, queue(kCtrK3, 0, nunits, true),
+  // ---- phase 3: K codes, newest units of phase 1 first.  Each unit's head
+  // k_mean row (512 B) arrives with it, in the slot's side buffer.
+  run(kBlockBytes, queue(kCtrK3, 0, nunits, true),
       [&](int u, uint8_t* dst, uint64_t* bar) {
         const uint32_t bytes = (uint32_t)unit_rows(u) * kHeadDim * 2;
-        mbar_arrive_expect_tx(bar, bytes + kHeadDim * 4);
+        mbar_arrive_expect_tx(bar, bytes + kSideBytes);
         bulk_load(dst, k + unit_in(u), bytes, bar, pol_first);
-        bulk_load(dst + kBlockBytes, k_mean + (size_t)(u / nblk) * kHeadDim, kHeadDim * 4, bar, pol_first);
+        bulk_load(side + (dst - ring) / kBlockBytes * kSideBytes, k_mean + (size_t)(u / nblk) * kHeadDim,
+                  kSideBytes, bar, pol_first);
       },
       [&](int u, const uint8_t* blk, bool ok, int par) -> bool {
         // every chunk of this thread starts at channel 8t mod 128
-        const float* mu = reinterpret_cast<const float*>(blk + kBlockBytes) + ((8 * t) & (kHeadDim - 1));
+        const float* mu = reinterpret_cast<const float*>(side + (blk - ring) / kBlockBytes * kSideBytes) +
+                          ((8 * t) & (kHeadDim - 1));
         float mr[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) mr[e] = mu[e];
