@@ -157,3 +157,43 @@ def test_every_key_corrected_is_exact_attention():
     print(f"\n[rho=1] vs exact FP64: {m}")
     assert m["cos"] >= 0.99999 and m["mean_rel"] <= 1e-4, m
     assert np.all(np.abs(got - ex) <= 1e-3 + 1e-4 * np.abs(ex))
+
+
+@pytest.mark.parametrize("layout", ["block_left_with_one_key", "first_and_last_keys_kept"])
+def test_patched_tiles_extreme_blocks(layout):
+    """The patched FP8 part (fewer than 64 corrected keys per head) at its
+    limits, with the key errors chosen by hand (the call takes them as input):
+    63 corrected keys in one 64-key block, so its single kept key (the last)
+    is copied 63 times; or 63 corrected keys spread over all four blocks, the
+    copied key being the block's first, or one in its middle, or after a
+    corrected first key.  Against the oracle with the same selection."""
+    fqa = _fqa()
+    w = dataclasses.replace(synth.workload(0), name="patch_extremes")      # B=1, H=2, N=256
+    g = synth.generate(w)
+    q, k, v = (U.to_device(g[t]) for t in "qkv")
+    qz, _ = fqa.quantize_keyerr(q, k, v)
+    N = w.N
+    err = np.zeros((w.B, w.H, N), np.float32)
+    if layout == "block_left_with_one_key":
+        err[:, :, 64:127] = 2.0                       # keys 64..126 of block 1; key 127 kept
+        rho = 63 / 256
+    else:
+        err[:, :, 0:16] = 2.0                         # block 0: copies key 16
+        err[:, :, 65:80] = 1.5                        # block 1: copies key 64
+        err[:, :, 128:144] = 3.0                      # block 2: copies key 144
+        err[:, :, 240:256] = 1.0                      # block 3: copies key 192; 16 + 15 + 16 + 16 = 63
+        rho = 63 / 256
+    kc = fqa.fqa_corrected_keys(N, rho)
+    assert kc == 63 and int((err > 0).sum(axis=2).max()) == 63
+    k_err = torch.from_numpy(err).cuda()
+    out32 = fqa.attention_fp8_corrected(q, k, v, qz, k_err, U.SCALE, rho, fqa.FQA_OUT_F32)
+    torch.cuda.synchronize()
+    assert fqa.fqa_debug_status()[0] == fqa.FQA_OK
+    oq = oracle.quantize(g["q"], g["k"], g["v"])
+    sel = oracle.select_keys(err, kc)
+    assert np.array_equal(sel.astype(bool), err > 0)
+    ref, amb = oracle.attention_fp8_corrected(g, oq, sel, U.SCALE, with_ambiguity=True)
+    got = out32.cpu().numpy().reshape(ref.shape).astype(np.float64)
+    m = U.metrics(got, ref)
+    assert m["mean_rel"] <= 2e-3, m
+    assert np.all(np.abs(got - ref) <= 1e-2 + amb), float((np.abs(got - ref) - amb).max())
