@@ -369,6 +369,18 @@ FQA_API fqa_status fqa_attention_nvfp4(const uint8_t* q4, const uint8_t* k4, con
 FQA_API fqa_status fqa_e2m1_encode(const float* x, uint8_t* out, size_t npairs, void* cuda_stream);
 
 /*
+ * fqa_exp2_error -- measures the exponential the attention kernels use for
+ * p = 2^(x - m) and the rescale factors (the hardware ex2 approximation with
+ * flush-to-zero) at every binary32 x in [lo, hi], -126 <= lo <= hi <= 0,
+ * against binary64 exp2 (results of 2^x below 2^-126 are skipped: they flush
+ * to zero by design).  *max_rel_bits (device, 4-byte aligned) receives the
+ * bit pattern of the largest relative error as a binary32 value; it is
+ * zeroed first.  A check of the error budget the parity tolerance assumes
+ * for this step (2^-21), not part of the path.
+ */
+FQA_API fqa_status fqa_exp2_error(float lo, float hi, uint32_t* max_rel_bits, void* cuda_stream);
+
+/*
  * fqa_e4m3_encode -- the library's binary32 -> E4M3 conversion (round to
  * nearest even, saturating to +-448, NaN -> 0x7F), exposed so that callers
  * can check the codec exhaustively.  x: FP32 [n], out: uint8 [n] (device).

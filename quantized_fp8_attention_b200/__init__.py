@@ -75,6 +75,8 @@ def _load():
     L.fqa_attention_nvfp4.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, ctypes.c_float, P, I, P]
     L.fqa_e2m1_encode.restype = I
     L.fqa_e2m1_encode.argtypes = [P, P, ctypes.c_size_t, P]
+    L.fqa_exp2_error.restype = I
+    L.fqa_exp2_error.argtypes = [ctypes.c_float, ctypes.c_float, P, P]
     _lib = L
     return L
 
@@ -224,6 +226,17 @@ def fqa_attention_nvfp4(q4, k4, sfq, sfk, sq1, sk1, v8, sv, sv_max, softmax_scal
 
 def fqa_e2m1_encode(x, out, stream=None) -> int:
     return _load().fqa_e2m1_encode(_ptr(x), _ptr(out), x.numel() // 2, _stream(stream))
+
+
+def fqa_exp2_error(lo: float, hi: float, max_rel_bits, stream=None) -> int:
+    return _load().fqa_exp2_error(float(lo), float(hi), _ptr(max_rel_bits), _stream(stream))
+
+
+def exp2_max_rel_error(lo: float, hi: float, device="cuda") -> float:
+    """Largest relative error of the kernels' exp2 over every binary32 in [lo, hi]."""
+    bits = torch.zeros(1, dtype=torch.int32, device=device)
+    _check(fqa_exp2_error(lo, hi, bits), "fqa_exp2_error")
+    return float(bits.cpu().view(torch.float32)[0])
 
 
 def fqa_debug_wait_timeout(limit_us: int, stream=None) -> int:

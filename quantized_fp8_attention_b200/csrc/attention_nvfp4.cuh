@@ -15,12 +15,16 @@
 // Organisation: the FP8 kernel's two Q tiles per CTA fill all 512 TMEM
 // columns, leaving none for the scale factors, so this kernel runs one
 // 128-row Q tile per work item (persistent, one CTA per SM):
-//   warps 0-3  softmax: thread = row = TMEM lane, all 128 keys of a tile; they
-//              also write the scale factors into TMEM (tcgen05.st) ahead of
-//              the MMAs that read them
-//   warp 4     TMA producer: Q (E2M1, 64 B rows, 64-byte swizzle) per item;
+//   warps 0-7  softmax: warp w handles TMEM lanes 32 (w % 4) .. and keys
+//              [64 hf, 64 hf + 64) of every tile, hf = w / 4 (two threads
+//              per row); each thread takes the row maximum from the raw
+//              maxima of both halves (read from TMEM), so the halves exchange
+//              only their row sums, once per item; warps 0-3 also write the
+//              scale factors into TMEM (tcgen05.st) ahead of the MMAs that
+//              read them
+//   warp 8     TMA producer: Q (E2M1, 64 B rows, 64-byte swizzle) per item;
 //              K (E2M1) and V (E4M3) tiles through three-stage rings
-//   warp 5     TMEM owner and single-thread MMA issuer
+//   warp 9     TMEM owner and single-thread MMA issuer
 // TMEM: S [0,128), O [128,256), SFA [256,264), SFB stage s [264+8s, 272+8s).
 // Scale-factor layout (per MMA of K = 64, 4 groups): the factor of row m and
 // group j sits in column base + m / 32, byte j, of lane m % 32, replicated in
@@ -33,8 +37,8 @@
 
 namespace fqa {
 
-constexpr int kNvThreads = 192;
-constexpr int kNvProducer = 4, kNvMma = 5;
+constexpr int kNvThreads = 320;
+constexpr int kNvProducer = 8, kNvMma = 9;
 
 struct NvTraits {
   static constexpr int kQKBytes = 128 * 64;                      // E2M1 tile, 128 rows x 64 B
@@ -44,10 +48,11 @@ struct NvTraits {
   static constexpr int kOffK = kOffQ + kQKBytes;
   static constexpr int kOffV = kOffK + kStages * kQKBytes;
   static constexpr int kOffP = kOffV + kStages * kVBytes;        // two buffers
-  static constexpr int kOffBar = kOffP + 2 * kVBytes;
+  static constexpr int kOffL = kOffP + 2 * kVBytes;               // [item parity][half][row] row sums
+  static constexpr int kOffBar = kOffL + 2 * 2 * 128 * 4;
   // fullK, fullV, emptyK, emptyV, barSFB [kStages]; barQ, barQfree, barSFA,
-  // barS, barSfree, barP, barPV, barDrain
-  static constexpr int kNumBars = 5 * kStages + 8;
+  // barS, barSfree, barP, barPV, barDrain, barL
+  static constexpr int kNumBars = 5 * kStages + 9;
   // more than half of the SM's 228 KB: one CTA per SM, so the 512-column TMEM
   // allocation never waits for a co-resident CTA
   static constexpr int kSmemUsed = kOffBar + 8 * kNumBars + 16 + 1024;
@@ -145,6 +150,8 @@ __global__ void __launch_bounds__(kNvThreads, 1)
   uint64_t* barP = barQ + 5;
   uint64_t* barPV = barQ + 6;
   uint64_t* barDrain = barQ + 7;
+  uint64_t* barL = barQ + 8;        // both halves' row sums of an item written
+  float* sL = reinterpret_cast<float*>(smem + T::kOffL);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + T::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -168,8 +175,9 @@ __global__ void __launch_bounds__(kNvThreads, 1)
     mbar_init(barQfree, 1);
     mbar_init(barSFA, kBlockM);
     mbar_init(barS, 1);
-    mbar_init(barSfree, kBlockM);
-    mbar_init(barP, kBlockM);
+    mbar_init(barSfree, 2 * kBlockM);
+    mbar_init(barP, 2 * kBlockM);
+    mbar_init(barL, 2 * kBlockM);
     mbar_init(barPV, 1);
     mbar_init(barDrain, 1);
     *abort_flag = 0;
@@ -282,12 +290,14 @@ __global__ void __launch_bounds__(kNvThreads, 1)
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------ softmax (warps 0-3)
-    const int r = threadIdx.x;                   // row of the tile == TMEM lane
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    // ------------------------------------------------ softmax (warps 0-7)
+    const int hf = warp >> 2;                    // keys [64 hf, 64 hf + 64) of each tile
+    const int r = threadIdx.x & 127;             // row of the tile == TMEM lane
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + T::kColS + lane_off, tO = tmem + T::kColO + lane_off;
     const uint32_t prow = smem_u32(sP) + (uint32_t)r * 128u;
     const uint32_t sw = (uint32_t)(r & 7);
+    const bool sf_writer = hf == 0;              // warps 0-3 write the scale factors
     // scale factors ride one step ahead of the MMAs that read them: the Q
     // factors of item it+1 go in once the last S MMA of item it completed
     // (before that S is released, so the MMA issuer never waits on a softmax
@@ -295,7 +305,7 @@ __global__ void __launch_bounds__(kNvThreads, 1)
     // stage was last read by tile g-2's MMA, which has completed)
     auto item_head = [&](int i) { return ((int)blockIdx.x + i * (int)gridDim.x) / nq; };
     auto item_qt = [&](int i) { return ((int)blockIdx.x + i * (int)gridDim.x) % nq; };
-    if (my_items > 0) {
+    if (sf_writer && my_items > 0) {
       write_scale_factors(tmem + T::kColSFA + lane_off, p.sfq,
                           (size_t)item_head(0) * N + (size_t)item_qt(0) * kBlockM, lane);
       write_scale_factors(tmem + T::kColSFB + lane_off, p.sfk, (size_t)item_head(0) * N, lane);
@@ -316,7 +326,7 @@ __global__ void __launch_bounds__(kNvThreads, 1)
       const float a_row = p.sq1[(size_t)head * nblk + qrow / 64];
       float m = -INFINITY, l = 0.0f;
       for (int j = 0; j < nkv; ++j, ++g) {
-        if (g + 1 < ntiles) {
+        if (sf_writer && g + 1 < ntiles) {
           // the next K tile: this item's tile j+1, or the next item's tile 0
           const size_t nrow = j + 1 < nkv ? hrow + (size_t)(j + 1) * kBlockN : (size_t)item_head(it + 1) * N;
           write_scale_factors(tmem + T::kColSFB + 8u * (uint32_t)((g + 1) % T::kStages) + lane_off, p.sfk,
@@ -327,11 +337,12 @@ __global__ void __launch_bounds__(kNvThreads, 1)
         }
         const float a0 = a_row * (__ldg(skp + 2 * j) * c_log2e);
         const float a1 = a_row * (__ldg(skp + 2 * j + 1) * c_log2e);
-        const float cpv0 = svmax > 0.0f ? 448.0f * (__ldg(svp + 2 * j) / svmax) : 0.0f;
-        const float cpv1 = svmax > 0.0f ? 448.0f * (__ldg(svp + 2 * j + 1) / svmax) : 0.0f;
+        const float ah = hf ? a1 : a0;
+        const float svh = __ldg(svp + 2 * j + hf);
+        const float cpv = svmax > 0.0f ? 448.0f * (svh / svmax) : 0.0f;
         if (!(ok = __all_sync(0xffffffffu, mbar_wait(barS, g & 1, abort_flag, p.status)))) break;
         tc_fence_after();
-        if (j == nkv - 1 && it + 1 < my_items) {
+        if (sf_writer && j == nkv - 1 && it + 1 < my_items) {
           // this item's last S MMA completed: the next item's Q factors
           write_scale_factors(tmem + T::kColSFA + lane_off, p.sfq,
                               (size_t)item_head(it + 1) * N + (size_t)item_qt(it + 1) * kBlockM, lane);
@@ -339,54 +350,64 @@ __global__ void __launch_bounds__(kNvThreads, 1)
           tc_fence_before();
           mbar_arrive(barSFA);
         }
-        float x[128];
-        float tmax = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t u[32];
-          tmem_ld32(tS + 32u * c, u);
+        // this half's 64 scores stay in registers; the other half's only give
+        // their raw maximum (a >= 0 and rounding is monotone, so the maximum
+        // of the rounded products is the rounded product of the raw maximum)
+        uint32_t u[64];
+        float mo;
+        {
+          uint32_t v[32];
+          tmem_ld32(tS + 64u * (uint32_t)hf, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+          tmem_ld32(tS + 64u * (uint32_t)hf + 32u, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+          tmem_ld32(tS + 64u * (uint32_t)(hf ^ 1), v);
           tmem_wait_ld();
-          const float a = c < 2 ? a0 : a1;
+          mo = __uint_as_float(v[0]);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            x[32 * c + e] = __fmul_rz(__uint_as_float(u[e]), a);
-            tmax = fmaxf(tmax, x[32 * c + e]);
-          }
+          for (int e = 1; e < 32; ++e) mo = fmaxf(mo, __uint_as_float(v[e]));
+          tmem_ld32(tS + 64u * (uint32_t)(hf ^ 1) + 32u, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) mo = fmaxf(mo, __uint_as_float(v[e]));
         }
         tc_fence_before();
         mbar_arrive(barSfree);                   // S may be overwritten by the next tile's MMA
-        const float m_new = fmaxf(m, tmax);
+        float mh = __uint_as_float(u[0]);
+#pragma unroll
+        for (int e = 1; e < 64; ++e) mh = fmaxf(mh, __uint_as_float(u[e]));
+        const float h0 = hf ? mo : mh, h1 = hf ? mh : mo;
+        const float m_new = fmaxf(m, fmaxf(__fmul_rz(h0, a0), __fmul_rz(h1, a1)));
         const float alpha = ex2_approx(m - m_new);
         float ls = 0.0f;
         const uint32_t pbuf = prow + (uint32_t)(g & 1) * T::kVBytes;
 #pragma unroll
-        for (int c16 = 0; c16 < 8; ++c16) {     // 16 keys: one 16-byte chunk of P
+        for (int c16 = 0; c16 < 4; ++c16) {     // 16 keys: one 16-byte chunk of P
           uint32_t pw[4];
-          const float cpv = c16 < 4 ? cpv0 : cpv1;
 #pragma unroll
           for (int w4 = 0; w4 < 4; ++w4) {
             float pv[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              pv[e] = ex2_approx(__fmaf_rn(x[16 * c16 + 4 * w4 + e], 1.0f, -m_new));
+              const float x = __fmul_rz(__uint_as_float(u[16 * c16 + 4 * w4 + e]), ah);
+              pv[e] = ex2_approx(__fmaf_rn(x, 1.0f, -m_new));
               ls += pv[e];
             }
             pw[w4] = e4m3x4(pv[0] * cpv, pv[1] * cpv, pv[2] * cpv, pv[3] * cpv);
           }
-          st_shared_v4(pbuf + (((uint32_t)c16 ^ sw) << 4), pw[0], pw[1], pw[2], pw[3]);
+          st_shared_v4(pbuf + ((((uint32_t)(4 * hf + c16)) ^ sw) << 4), pw[0], pw[1], pw[2], pw[3]);
         }
         if (j > 0) {
           if (!(ok = __all_sync(0xffffffffu, mbar_wait(barPV, (g - 1) & 1, abort_flag, p.status)))) break;
           tc_fence_after();
           if (__any_sync(0xffffffffu, m_new != m)) {
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < 2; ++c) {
               uint32_t o[32];
-              tmem_ld32(tO + 32u * c, o);
+              const uint32_t col = 64u * (uint32_t)hf + 32u * (uint32_t)c;
+              tmem_ld32(tO + col, o);
               tmem_wait_ld();
 #pragma unroll
               for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-              tmem_st32(tO + 32u * c, o);
+              tmem_st32(tO + col, o);
             }
             tmem_wait_st();
           }
@@ -398,37 +419,45 @@ __global__ void __launch_bounds__(kNvThreads, 1)
         mbar_arrive(barP);
       }
       if (!ok) break;
-      // ------------------------------------------------ epilogue
+      // ------------------------------------------------ epilogue: this half's 64 columns
+      float* lx = sL + (it & 1) * 2 * 128;
+      lx[hf * 128 + r] = l;
+      mbar_arrive(barL);
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(barL, it & 1, abort_flag, p.status)))) break;
+      const float l_row = lx[r] + lx[128 + r];
       if (!(ok = __all_sync(0xffffffffu, mbar_wait(barPV, (g - 1) & 1, abort_flag, p.status)))) break;
       tc_fence_after();
-      const float fin = (svmax / 448.0f) / l;
+      const float fin = (svmax / 448.0f) / l_row;
       const size_t orow = hrow + (size_t)qrow;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t o[32];
-        tmem_ld32(tO + 32u * c, o);
+        const int col = 64 * hf + 32 * c;
+        tmem_ld32(tO + (uint32_t)col, o);
         tmem_wait_ld();
         if (p.out_f32) {
-          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow * 128 + 32 * c);
+          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow * 128 + col);
 #pragma unroll
           for (int e = 0; e < 8; ++e)
             dst[e] = make_float4(__uint_as_float(o[4 * e]) * fin, __uint_as_float(o[4 * e + 1]) * fin,
                                  __uint_as_float(o[4 * e + 2]) * fin, __uint_as_float(o[4 * e + 3]) * fin);
         } else {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + orow * 128 + 32 * c);
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + orow * 128 + col);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             uint32_t w4[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(o[8 * e + 2 * u]) * fin,
-                                                              __uint_as_float(o[8 * e + 2 * u + 1]) * fin);
-              w4[u] = *reinterpret_cast<const uint32_t*>(&b2);
+            for (int q = 0; q < 4; ++q) {
+              const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(o[8 * e + 2 * q]) * fin,
+                                                              __uint_as_float(o[8 * e + 2 * q + 1]) * fin);
+              w4[q] = *reinterpret_cast<const uint32_t*>(&b2);
             }
             dst[e] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
           }
         }
       }
+      // the next item's first PV overwrites O only after this warp's next
+      // barP arrival, which comes after these loads
       tc_fence_before();
     }
   }

@@ -573,6 +573,22 @@ fqa_status fqa_e2m1_encode(const float* x, uint8_t* out, size_t npairs, void* cu
   return launch_status();
 }
 
+fqa_status fqa_exp2_error(float lo, float hi, uint32_t* max_rel_bits, void* cuda_stream) {
+  if (max_rel_bits == nullptr) return FQA_ERR_INVALID_ARG;
+  if (!(lo <= hi) || !(hi <= 0.0f) || !(lo >= -126.0f)) return FQA_ERR_INVALID_ARG;
+  if (!aligned(max_rel_bits, 4)) return FQA_ERR_MISALIGNED;
+  // negative binary32 values from hi down to lo are consecutive bit patterns
+  uint32_t hb, lb;
+  const float h = hi == 0.0f ? -0.0f : hi;
+  std::memcpy(&hb, &h, 4);
+  std::memcpy(&lb, &lo, 4);
+  const uint32_t n = lb - hb + 1;
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  if (cudaMemsetAsync(max_rel_bits, 0, 4, s) != cudaSuccess) return FQA_ERR_CUDA;
+  exp2_error_kernel<<<148 * 16, 256, 0, s>>>(lb, n, reinterpret_cast<unsigned int*>(max_rel_bits));
+  return launch_status();
+}
+
 fqa_status fqa_e4m3_encode(const float* x, uint8_t* out, size_t n, void* cuda_stream) {
   if (x == nullptr || out == nullptr) return FQA_ERR_INVALID_ARG;
   if (n == 0) return FQA_OK;

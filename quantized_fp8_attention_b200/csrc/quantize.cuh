@@ -474,6 +474,23 @@ __global__ void wait_timeout_kernel(uint32_t* status, uint64_t limit_ns) {
   mbar_wait_limit(&bar, 0, &abort_flag, status, limit_ns);
 }
 
+// The exponential every attention kernel uses (ex2.approx.ftz.f32) at every
+// binary32 x in [lo, hi] (lo <= hi <= 0 here), against binary64 exp2: the
+// largest relative error, as its bit pattern (non-negative floats order like
+// their bits), into *max_rel_bits.
+__global__ void exp2_error_kernel(uint32_t lo_bits, uint32_t n, unsigned int* max_rel_bits) {
+  float worst = 0.0f;
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    // negative floats: larger magnitude <-> larger bit pattern; walk from hi down to lo
+    const float x = __uint_as_float(lo_bits - i);
+    const float y = ex2_approx(x);
+    const double ref = exp2((double)x);
+    if (ref >= 0x1p-126) worst = fmaxf(worst, (float)(fabs((double)y - ref) / ref));
+  }
+  for (int o = 16; o > 0; o >>= 1) worst = fmaxf(worst, __shfl_xor_sync(0xffffffffu, worst, o));
+  if ((threadIdx.x & 31) == 0) atomicMax(max_rel_bits, __float_as_uint(worst));
+}
+
 // Standalone conversion kernel: every binary32 input -> its E4M3 code via the
 // same instruction the quantizer uses (for exhaustive codec checks).
 __global__ void e4m3_encode_kernel(const float* __restrict__ x, uint8_t* __restrict__ out, size_t n) {

@@ -164,3 +164,14 @@ def test_nvfp4_validation(L):
     assert attn(sv=_p(0x10002)) == 3
     assert L.fqa_e2m1_encode(None, ok, 4, None) == 1
     assert L.fqa_e2m1_encode(_p(0x10004), ok, 4, None) == 3
+
+
+def test_exp2_error_validation(L):
+    ok = _p(0x10000)
+    f = ctypes.c_float
+    L.fqa_exp2_error.argtypes = [f, f, P, P]
+    assert L.fqa_exp2_error(f(-30.0), f(0.0), None, None) == 1
+    assert L.fqa_exp2_error(f(0.0), f(-30.0), ok, None) == 1        # lo > hi
+    assert L.fqa_exp2_error(f(-30.0), f(1.0), ok, None) == 1        # hi > 0
+    assert L.fqa_exp2_error(f(-200.0), f(0.0), ok, None) == 1       # lo < -126
+    assert L.fqa_exp2_error(f(-30.0), f(0.0), _p(0x10002), None) == 3

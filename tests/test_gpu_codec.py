@@ -27,3 +27,17 @@ def test_e4m3_encode_exhaustive():
             got, ref = got[~nan], ref[~nan]
         bad = np.count_nonzero(got != ref)
         assert bad == 0, f"chunk {c}: {bad} codes differ"
+
+
+def test_kernel_exp2_within_the_parity_bound():
+    """The exponential of every attention kernel (p = 2^(x - m), the rescale
+    factors) against binary64 exp2 at every binary32 x in [-30, 0] -- the
+    range where a P code can be nonzero (p * 448 >= 2^-10 needs x - m >= -19)
+    and where a term can move the row sum by more than 2^-30 of its largest
+    term.  The oracle's ambiguity bound assumes a relative error of at most
+    2^-21 for this step; this measures it."""
+    import quantized_fp8_attention_b200 as fqa
+    err = fqa.exp2_max_rel_error(-30.0, 0.0)
+    print(f"\nmax relative error of the kernels' exp2 on [-30, 0]: {err:.3e} (2^{np.log2(err):.2f})")
+    assert 0.0 < err <= 2.0 ** -21
+    assert fqa.fqa_debug_status()[0] == fqa.FQA_OK
