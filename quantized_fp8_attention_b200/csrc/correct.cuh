@@ -41,12 +41,20 @@ namespace fqa {
 // ------------------------------------------------------------ selection
 
 constexpr int kSelThreads = 1024;
+constexpr int kSelStageMax = 32768;   // heads up to this length are staged in shared memory (128 KB)
 
 __global__ void __launch_bounds__(kSelThreads, 1)
     select_keys_kernel(const float* __restrict__ err, int N, int kc, uint32_t* __restrict__ kmask,
-                       int* __restrict__ idx) {
+                       int* __restrict__ idx, int staged) {
+  extern __shared__ uint32_t sel_stage[];
   const int bh = blockIdx.x, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-  const uint32_t* e = reinterpret_cast<const uint32_t*>(err) + (size_t)bh * N;
+  const uint32_t* eg = reinterpret_cast<const uint32_t*>(err) + (size_t)bh * N;
+  // the head's errors, read five times below: from shared memory when they fit
+  if (staged) {
+    for (int i = tid; i < N; i += kSelThreads) sel_stage[i] = __ldg(eg + i);
+    __syncthreads();
+  }
+  const uint32_t* e = staged ? sel_stage : eg;
   const int nw = (N + 31) / 32;
   uint32_t* km = kmask + (size_t)bh * nw;
   int* id = idx + (size_t)bh * (size_t)kc;
@@ -68,22 +76,41 @@ __global__ void __launch_bounds__(kSelThreads, 1)
     __syncthreads();
     const uint32_t prefix = s_prefix, mask = s_mask;
     for (int i = tid; i < N; i += kSelThreads) {
-      const uint32_t u = __ldg(e + i);
+      const uint32_t u = e[i];
       if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
     }
     __syncthreads();
-    if (tid == 0) {
-      int want = s_want, cum = 0, digit = 0;
-      for (int b = 255; b >= 0; --b) {
-        if (cum + (int)hist[b] >= want) {
-          digit = b;
-          break;
-        }
-        cum += (int)hist[b];
+    if (wid == 0) {
+      // the digit: walking the bins from 255 down, the first where the count
+      // so far reaches `want`; lane l holds bins 255 - 8l .. 248 - 8l
+      const int want = s_want;
+      int c[8], tot = 0;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        c[q] = (int)hist[255 - 8 * lane - q];
+        tot += c[q];
       }
-      s_want = want - cum;                      // still needed among this digit
-      s_prefix = prefix | ((uint32_t)digit << shift);
-      s_mask = mask | (255u << shift);
+      int incl = tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const uint32_t hit = __ballot_sync(0xffffffffu, incl >= want);
+      if (lane == __ffs(hit) - 1) {
+        int cum = incl - tot, digit = 255 - 8 * lane;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          if (cum + c[q] >= want) {
+            digit = 255 - 8 * lane - q;
+            break;
+          }
+          cum += c[q];
+        }
+        s_want = want - cum;                    // still needed among this digit
+        s_prefix = prefix | ((uint32_t)digit << shift);
+        s_mask = mask | (255u << shift);
+      }
     }
     __syncthreads();
   }
@@ -98,7 +125,7 @@ __global__ void __launch_bounds__(kSelThreads, 1)
   __syncthreads();
   for (int base = 0; base < N; base += kSelThreads) {
     const int i = base + tid;
-    const uint32_t u = i < N ? __ldg(e + i) : 0u;
+    const uint32_t u = i < N ? e[i] : 0u;
     const bool gt = i < N && u > T, eq = i < N && u == T;
     const uint32_t lt_mask = (1u << lane) - 1u;
     const uint32_t beq = __ballot_sync(0xffffffffu, eq);
@@ -566,7 +593,6 @@ __global__ void __launch_bounds__(kCorrThreads, CorrTraits<kKeys>::kCtasPerSm)
       const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
       const bool store = qrow < N && ok;
       float w1 = 0.0f, w2 = 0.0f, inv = 0.0f, l1 = 0.0f;
-      const float* o1r = p.o1 + (hbase + (size_t)(qrow < N ? qrow : 0)) * 128;
       if (store) {
         const float2 st = p.stats[hbase + qrow];
         l1 = st.y;
@@ -577,49 +603,67 @@ __global__ void __launch_bounds__(kCorrThreads, CorrTraits<kKeys>::kCtasPerSm)
         inv = L > 0.0f ? 1.0f / L : 0.0f;
       }
       const float a1 = (p.o1_raw ? w1 : l1 * w1) * inv, a2 = w2 * inv;
-#pragma unroll 1
-      for (int c2 = 0; c2 < 4; c2 += 2) {
-        // two 32-column chunks per round trip: both halves' O1 loads in flight
-        float4 f1[16];
-        if (store) {
-          const float4* s1 = reinterpret_cast<const float4*>(o1r + 32 * c2);
+      // the FP8 part's rows come in through shared memory (the P buffers are
+      // free once PV completed): the warp loads its 32 rows 32 columns at a
+      // time with coalesced 16-byte accesses (8 lanes per 128-byte row
+      // segment), then each thread reads its own row; two staging buffers let
+      // the next chunk's loads fly while this one is merged
+      const int wrow0 = tq * 128 + 32 * warp;
+      uint8_t* stg_buf[2] = {sPhi + warp * 4096, sPlo + warp * 4096};
+      float4 nxt[8];
+      auto load_chunk = [&](int c) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) f1[e] = __ldg(s1 + e);
+        for (int i = 0; i < 8; ++i) {
+          const int grow = wrow0 + 4 * i + (lane >> 3);
+          nxt[i] = (ok && grow < N)
+                       ? __ldg(reinterpret_cast<const float4*>(p.o1 + (hbase + (size_t)grow) * 128 + 32 * c) + (lane & 7))
+                       : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
         }
+      };
+      load_chunk(0);
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint8_t* stg = stg_buf[c & 1];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int c = c2 + h;
-          uint32_t o[32];
-          tmem_ld32(tmem + 128u + lane_off + 32u * c, o);
-          tmem_wait_ld();
-          if (!store) continue;
-          float res[32];
+        for (int i = 0; i < 8; ++i) {
+          const int rr = 4 * i + (lane >> 3), q = lane & 7;
+          *reinterpret_cast<float4*>(stg + rr * 128 + ((q ^ (rr & 7)) << 4)) = nxt[i];
+        }
+        if (c + 1 < 4) load_chunk(c + 1);          // in flight during this chunk's merge
+        __syncwarp();
+        float4 f1[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float4 f = f1[8 * h + e];
-            res[4 * e] = f.x * a1 + __uint_as_float(o[4 * e]) * a2;
-            res[4 * e + 1] = f.y * a1 + __uint_as_float(o[4 * e + 1]) * a2;
-            res[4 * e + 2] = f.z * a1 + __uint_as_float(o[4 * e + 2]) * a2;
-            res[4 * e + 3] = f.w * a1 + __uint_as_float(o[4 * e + 3]) * a2;
-          }
-          const size_t orow = hbase + qrow;
-          if (p.out_f32) {
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow * 128 + 32 * c);
+        for (int q = 0; q < 8; ++q) f1[q] = *reinterpret_cast<const float4*>(stg + lane * 128 + ((q ^ (lane & 7)) << 4));
+        uint32_t o[32];
+        tmem_ld32(tmem + 128u + lane_off + 32u * c, o);
+        tmem_wait_ld();
+        if (!store) continue;
+        float res[32];
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-              dst[e] = make_float4(res[4 * e], res[4 * e + 1], res[4 * e + 2], res[4 * e + 3]);
-          } else {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + orow * 128 + 32 * c);
+        for (int e = 0; e < 8; ++e) {
+          const float4 f = f1[e];
+          res[4 * e] = f.x * a1 + __uint_as_float(o[4 * e]) * a2;
+          res[4 * e + 1] = f.y * a1 + __uint_as_float(o[4 * e + 1]) * a2;
+          res[4 * e + 2] = f.z * a1 + __uint_as_float(o[4 * e + 2]) * a2;
+          res[4 * e + 3] = f.w * a1 + __uint_as_float(o[4 * e + 3]) * a2;
+        }
+        const size_t orow = hbase + qrow;
+        if (p.out_f32) {
+          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow * 128 + 32 * c);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              uint32_t w4[4];
+          for (int e = 0; e < 8; ++e)
+            dst[e] = make_float4(res[4 * e], res[4 * e + 1], res[4 * e + 2], res[4 * e + 3]);
+        } else {
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + orow * 128 + 32 * c);
 #pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                const __nv_bfloat162 b2 = __floats2bfloat162_rn(res[8 * e + 2 * u], res[8 * e + 2 * u + 1]);
-                w4[u] = *reinterpret_cast<const uint32_t*>(&b2);
-              }
-              dst[e] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          for (int e = 0; e < 4; ++e) {
+            uint32_t w4[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const __nv_bfloat162 b2 = __floats2bfloat162_rn(res[8 * e + 2 * u], res[8 * e + 2 * u + 1]);
+              w4[u] = *reinterpret_cast<const uint32_t*>(&b2);
             }
+            dst[e] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
           }
         }
       }

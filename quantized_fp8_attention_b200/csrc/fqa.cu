@@ -410,8 +410,13 @@ fqa_status fqa_select_keys(const float* k_err, int B, int H, int N, int kc, uint
   for (const void* p : a4)
     if (!aligned(p, 4)) return FQA_ERR_MISALIGNED;
   if (!status_ptr(&st)) return st;
-  select_keys_kernel<<<B * H, kSelThreads, 0, static_cast<cudaStream_t>(cuda_stream)>>>(k_err, N, kc, kmask,
-                                                                                      idx);
+  const int staged = N <= kSelStageMax ? 1 : 0;
+  const int smem = staged ? N * 4 : 0;
+  if (staged && cudaFuncSetAttribute(select_keys_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     kSelStageMax * 4) != cudaSuccess)
+    return FQA_ERR_CUDA;
+  select_keys_kernel<<<B * H, kSelThreads, smem, static_cast<cudaStream_t>(cuda_stream)>>>(k_err, N, kc, kmask,
+                                                                                         idx, staged);
   return launch_status();
 }
 
