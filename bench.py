@@ -223,15 +223,13 @@ def run_sweep(args):
         cws = fqa.alloc_corrected_workspace(w.B, w.H, w.N, 0.005, dev)
         ms_c = timed(lambda: fqa.attention_fp8_corrected(q, k, v, qz, k_err, scale, 0.005, fqa.FQA_OUT_BF16,
                                                          out=out, workspace=cws), reps(1000))
-        # NVFP4 Q.K (N a multiple of 128): the FP4 quantizer and the attention
-        nv = None
-        if w.N % 128 == 0:
-            fqa.quantize(q, k, v, out=qz, workspace=ws)
-            qn = fqa.quantize_nvfp4_qk(q, k, qz.k_mean)
-            ms_n = timed(lambda: fqa.attention_nvfp4(qn, qz, scale, fqa.FQA_OUT_BF16, out=out), reps(650))
-            ms_nq = timed(lambda: fqa.quantize_nvfp4_qk(q, k, qz.k_mean, out=qn), 100, pre=lambda: flush.fill_(1))
-            nv = {"ms": ms_n, "tflops": w.flops / ms_n / 1e9, "time_vs_fp8": ms_n / ms_a,
-                  "quantize_nvfp4_qk_ms": ms_nq}
+        # NVFP4 Q.K: the FP4 quantizer and the attention
+        fqa.quantize(q, k, v, out=qz, workspace=ws)
+        qn = fqa.quantize_nvfp4_qk(q, k, qz.k_mean)
+        ms_n = timed(lambda: fqa.attention_nvfp4(qn, qz, scale, fqa.FQA_OUT_BF16, out=out), reps(850))
+        ms_nq = timed(lambda: fqa.quantize_nvfp4_qk(q, k, qz.k_mean, out=qn), 100, pre=lambda: flush.fill_(1))
+        nv = {"ms": ms_n, "tflops": w.flops / ms_n / 1e9, "time_vs_fp8": ms_n / ms_a,
+              "quantize_nvfp4_qk_ms": ms_nq}
         st, flags = fqa.fqa_debug_status()
         if st != fqa.FQA_OK:
             raise RuntimeError(f"device status {flags:#x} on {w.name}")
@@ -329,10 +327,8 @@ def accuracy_sample(w, g, q, k, v, scale, rho, qz, k_err, out, cws):
     plain = cos(fqa.attention_fp8(qz, scale, fqa.FQA_OUT_F32))
     fqa.quantize_keyerr(q, k, v, out=qz, k_err=k_err)
     corr = cos(fqa.attention_fp8_corrected(q, k, v, qz, k_err, scale, rho, fqa.FQA_OUT_F32, workspace=cws))
-    nv = None
-    if w.N % 128 == 0:
-        fqa.quantize(q, k, v, out=qz)
-        nv = cos(fqa.attention_nvfp4(fqa.quantize_nvfp4_qk(q, k, qz.k_mean), qz, scale, fqa.FQA_OUT_F32))
+    fqa.quantize(q, k, v, out=qz)
+    nv = cos(fqa.attention_nvfp4(fqa.quantize_nvfp4_qk(q, k, qz.k_mean), qz, scale, fqa.FQA_OUT_F32))
     sample = f"heads {heads}, rows [0,128) u [N/2, N/2+128) u [N-128, N), all keys"
     accuracy = {"cos_vs_exact_fp64": plain, "target": 0.995, "meets_target": plain >= 0.995, "sample": sample}
     corrected = {"rho": rho, "keys_per_head": fqa.fqa_corrected_keys(w.N, rho), "cos_vs_exact_fp64": corr,
@@ -554,27 +550,25 @@ def run_fqa(args, rank: int, world: int):
 
     # NVFP4 Q.K with FP8 P.V, same inputs: the FP8 quantizer (V codes and the K
     # mean), the NVFP4 quantizer of Q and smoothed K, the attention
-    nv_ms = None
-    if N % 128 == 0:
-        qn = fqa.alloc_quantized_nvfp4(B, H, N, dev)
+    qn = fqa.alloc_quantized_nvfp4(B, H, N, dev)
 
-        def nvfp4_step():
-            fqa.quantize(q, k, v, out=qz, workspace=ws)
-            fqa.quantize_nvfp4_qk(q, k, qz.k_mean, out=qn)
-            fqa.attention_nvfp4(qn, qz, scale, fqa.FQA_OUT_BF16, out=out)
+    def nvfp4_step():
+        fqa.quantize(q, k, v, out=qz, workspace=ws)
+        fqa.quantize_nvfp4_qk(q, k, qz.k_mean, out=qn)
+        fqa.attention_nvfp4(qn, qz, scale, fqa.FQA_OUT_BF16, out=out)
 
-        for _ in range(3):
-            nvfp4_step()
-        Kn = max(1, K // 4)
-        e0.record(stream)
-        for _ in range(Kn):
-            nvfp4_step()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        nv_ms = e0.elapsed_time(e1) / Kn
-        st, flags = fqa.fqa_debug_status()
-        if st != fqa.FQA_OK:
-            raise RuntimeError(f"device status {flags:#x} after the NVFP4 steps")
+    for _ in range(3):
+        nvfp4_step()
+    Kn = max(1, K // 4)
+    e0.record(stream)
+    for _ in range(Kn):
+        nvfp4_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    nv_ms = e0.elapsed_time(e1) / Kn
+    st, flags = fqa.fqa_debug_status()
+    if st != fqa.FQA_OK:
+        raise RuntimeError(f"device status {flags:#x} after the NVFP4 steps")
 
     ulysses = run_ulysses(w0, scale, dev, rank, world, K, ms_per_step) if world > 1 else None
 
@@ -591,10 +585,9 @@ def run_fqa(args, rank: int, world: int):
                      clk.summary(), probe, cpu, traffic_per_launch(), pk, pk_kind, corrected, accuracy)
     if ulysses is not None:
         line["ulysses"] = ulysses
-    if nv_ms is not None:
-        line["nvfp4"] = {"ms_per_step": nv_ms, "tflops": flops / (nv_ms * 1e-3) / 1e12,
-                         "step": "fqa_quantize + fqa_quantize_nvfp4_qk + fqa_attention_nvfp4",
-                         "time_vs_fp8_step": nv_ms / ms_per_step, "cos_vs_exact_fp64": nv_cos}
+    line["nvfp4"] = {"ms_per_step": nv_ms, "tflops": flops / (nv_ms * 1e-3) / 1e12,
+                     "step": "fqa_quantize + fqa_quantize_nvfp4_qk + fqa_attention_nvfp4",
+                     "time_vs_fp8_step": nv_ms / ms_per_step, "cos_vs_exact_fp64": nv_cos}
     print(json.dumps(line), flush=True)
 
 

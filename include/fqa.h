@@ -352,7 +352,8 @@ FQA_API fqa_status fqa_quantize_nvfp4_qk(const void* q, const void* k, const flo
  * FP32, out = O * (sv_max / 448) / l.
  * q4 .. sk1: fqa_quantize_nvfp4_qk() outputs; v8, sv, sv_max: fqa_quantize()
  * outputs.  q4, k4, v8 and out 16-byte aligned, sfq and sfk 8-byte aligned.
- * N must be a multiple of 128 (FQA_ERR_UNSUPPORTED otherwise).
+ * Any N >= 1: the last 128-key tile of a short sequence holds N % 128 keys
+ * (keys past N take no part), as in fqa_attention_fp8().
  */
 FQA_API fqa_status fqa_attention_nvfp4(const uint8_t* q4, const uint8_t* k4, const uint8_t* sfq,
                                        const uint8_t* sfk, const float* sq1, const float* sk1,

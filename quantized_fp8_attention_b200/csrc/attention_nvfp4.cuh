@@ -113,18 +113,26 @@ struct NvParams {
 // This thread's lane of the scale factors of 128 rows starting at `row0`
 // (sf: [rows][8] bytes): column (4 kk + m / 32) gets the four factors of MMA
 // kk of row 32 (m / 32) + lane, so the four lane quarters hold identical
-// copies.
-__device__ __forceinline__ void write_scale_factors(uint32_t taddr, const uint8_t* sf, size_t row0, int lane) {
+// copies.  Rows at or past `rend` (beyond the end of the sequence) get zero
+// factors and are not read.
+__device__ __forceinline__ void write_scale_factors(uint32_t taddr, const uint8_t* sf, size_t row0, size_t rend,
+                                                    int lane) {
   uint32_t v[8];
 #pragma unroll
   for (int mh = 0; mh < 4; ++mh) {
-    const uint2 f = __ldg(reinterpret_cast<const uint2*>(sf + (row0 + 32 * mh + lane) * 8));
+    const size_t row = row0 + 32 * mh + lane;
+    const uint2 f = row < rend ? __ldg(reinterpret_cast<const uint2*>(sf + row * 8)) : make_uint2(0u, 0u);
     v[mh] = f.x;
     v[4 + mh] = f.y;
   }
   tmem_st8(taddr, v);
 }
 
+// kShortTail: N is not a multiple of 128 -- the last Q tile and the last KV
+// tile are short: keys past N get x = -inf (no maximum, p or row-sum term;
+// their V rows are zero-filled by the tensor map), rows past N are not
+// stored.  Aligned calls use kShortTail = false and carry none of that code.
+template <bool kShortTail>
 __global__ void __launch_bounds__(kNvThreads, 1)
     attn_nvfp4_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const NvParams p) {
@@ -156,8 +164,9 @@ __global__ void __launch_bounds__(kNvThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int N = p.N, nkv = N / kBlockN, nblk = N / 64;
-  const int nq = N / kBlockM;
+  const int N = p.N, nkv = (N + kBlockN - 1) / kBlockN, nblk = (N + 63) / 64;
+  const int nq = (N + kBlockM - 1) / kBlockM;
+  const int valid_last = N - (nkv - 1) * kBlockN;   // keys in the last KV tile
   const int nitems = p.B * p.H * nq;
   const int my_items = nitems > (int)blockIdx.x ? (nitems - 1 - (int)blockIdx.x) / gridDim.x + 1 : 0;
   const int ntiles = my_items * nkv;
@@ -306,9 +315,9 @@ __global__ void __launch_bounds__(kNvThreads, 1)
     auto item_head = [&](int i) { return ((int)blockIdx.x + i * (int)gridDim.x) / nq; };
     auto item_qt = [&](int i) { return ((int)blockIdx.x + i * (int)gridDim.x) % nq; };
     if (sf_writer && my_items > 0) {
-      write_scale_factors(tmem + T::kColSFA + lane_off, p.sfq,
-                          (size_t)item_head(0) * N + (size_t)item_qt(0) * kBlockM, lane);
-      write_scale_factors(tmem + T::kColSFB + lane_off, p.sfk, (size_t)item_head(0) * N, lane);
+      const size_t h0 = (size_t)item_head(0) * N;
+      write_scale_factors(tmem + T::kColSFA + lane_off, p.sfq, h0 + (size_t)item_qt(0) * kBlockM, h0 + N, lane);
+      write_scale_factors(tmem + T::kColSFB + lane_off, p.sfk, h0, h0 + N, lane);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(barSFA);
@@ -323,29 +332,37 @@ __global__ void __launch_bounds__(kNvThreads, 1)
       const float* skp = p.sk1 + (size_t)head * nblk;
       const float* svp = p.sv + (size_t)head * nblk;
       const float svmax = p.sv_max[head];
-      const float a_row = p.sq1[(size_t)head * nblk + qrow / 64];
+      const float a_row = p.sq1[(size_t)head * nblk + min(qrow, N - 1) / 64];
+      // block scales of a tile; blocks past the end of a short sequence are
+      // read clamped (their keys are absent)
+      auto blk = [nblk](int J) { return (kShortTail && J >= nblk) ? nblk - 1 : J; };
       float m = -INFINITY, l = 0.0f;
       for (int j = 0; j < nkv; ++j, ++g) {
         if (sf_writer && g + 1 < ntiles) {
           // the next K tile: this item's tile j+1, or the next item's tile 0
-          const size_t nrow = j + 1 < nkv ? hrow + (size_t)(j + 1) * kBlockN : (size_t)item_head(it + 1) * N;
+          const size_t nh = j + 1 < nkv ? hrow : (size_t)item_head(it + 1) * N;
+          const size_t nrow = j + 1 < nkv ? hrow + (size_t)(j + 1) * kBlockN : nh;
           write_scale_factors(tmem + T::kColSFB + 8u * (uint32_t)((g + 1) % T::kStages) + lane_off, p.sfk,
-                              nrow, lane);
+                              nrow, nh + N, lane);
           tmem_wait_st();
           tc_fence_before();
           mbar_arrive(&barSFB[(g + 1) % T::kStages]);
         }
         const float a0 = a_row * (__ldg(skp + 2 * j) * c_log2e);
-        const float a1 = a_row * (__ldg(skp + 2 * j + 1) * c_log2e);
+        const float a1 = a_row * (__ldg(skp + blk(2 * j + 1)) * c_log2e);
         const float ah = hf ? a1 : a0;
-        const float svh = __ldg(svp + 2 * j + hf);
+        const float svh = __ldg(svp + blk(2 * j + hf));
+        // keys of this half present in the tile (all but in a short last tile)
+        const int nvh = (kShortTail && j == nkv - 1) ? min(64, max(0, valid_last - 64 * hf)) : 64;
+        const int nvo = (kShortTail && j == nkv - 1) ? min(64, max(0, valid_last - 64 * (hf ^ 1))) : 64;
         const float cpv = svmax > 0.0f ? 448.0f * (svh / svmax) : 0.0f;
         if (!(ok = __all_sync(0xffffffffu, mbar_wait(barS, g & 1, abort_flag, p.status)))) break;
         tc_fence_after();
         if (sf_writer && j == nkv - 1 && it + 1 < my_items) {
           // this item's last S MMA completed: the next item's Q factors
-          write_scale_factors(tmem + T::kColSFA + lane_off, p.sfq,
-                              (size_t)item_head(it + 1) * N + (size_t)item_qt(it + 1) * kBlockM, lane);
+          const size_t nh = (size_t)item_head(it + 1) * N;
+          write_scale_factors(tmem + T::kColSFA + lane_off, p.sfq, nh + (size_t)item_qt(it + 1) * kBlockM, nh + N,
+                              lane);
           tmem_wait_st();
           tc_fence_before();
           mbar_arrive(barSFA);
@@ -361,21 +378,27 @@ __global__ void __launch_bounds__(kNvThreads, 1)
           tmem_ld32(tS + 64u * (uint32_t)hf + 32u, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
           tmem_ld32(tS + 64u * (uint32_t)(hf ^ 1), v);
           tmem_wait_ld();
-          mo = __uint_as_float(v[0]);
+          mo = -INFINITY;
 #pragma unroll
-          for (int e = 1; e < 32; ++e) mo = fmaxf(mo, __uint_as_float(v[e]));
+          for (int e = 0; e < 32; ++e)
+            if (!kShortTail || e < nvo) mo = fmaxf(mo, __uint_as_float(v[e]));
           tmem_ld32(tS + 64u * (uint32_t)(hf ^ 1) + 32u, v);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) mo = fmaxf(mo, __uint_as_float(v[e]));
+          for (int e = 0; e < 32; ++e)
+            if (!kShortTail || 32 + e < nvo) mo = fmaxf(mo, __uint_as_float(v[e]));
         }
         tc_fence_before();
         mbar_arrive(barSfree);                   // S may be overwritten by the next tile's MMA
-        float mh = __uint_as_float(u[0]);
+        float mh = -INFINITY;
 #pragma unroll
-        for (int e = 1; e < 64; ++e) mh = fmaxf(mh, __uint_as_float(u[e]));
+        for (int e = 0; e < 64; ++e)
+          if (!kShortTail || e < nvh) mh = fmaxf(mh, __uint_as_float(u[e]));
         const float h0 = hf ? mo : mh, h1 = hf ? mh : mo;
-        const float m_new = fmaxf(m, fmaxf(__fmul_rz(h0, a0), __fmul_rz(h1, a1)));
+        // (a half with no key present has raw maximum -inf: it takes no part)
+        const float x0 = (kShortTail && h0 == -INFINITY) ? -INFINITY : __fmul_rz(h0, a0);
+        const float x1 = (kShortTail && h1 == -INFINITY) ? -INFINITY : __fmul_rz(h1, a1);
+        const float m_new = fmaxf(m, fmaxf(x0, x1));
         const float alpha = ex2_approx(m - m_new);
         float ls = 0.0f;
         const uint32_t pbuf = prow + (uint32_t)(g & 1) * T::kVBytes;
@@ -388,7 +411,7 @@ __global__ void __launch_bounds__(kNvThreads, 1)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const float x = __fmul_rz(__uint_as_float(u[16 * c16 + 4 * w4 + e]), ah);
-              pv[e] = ex2_approx(__fmaf_rn(x, 1.0f, -m_new));
+              pv[e] = (kShortTail && 16 * c16 + 4 * w4 + e >= nvh) ? 0.0f : ex2_approx(__fmaf_rn(x, 1.0f, -m_new));
               ls += pv[e];
             }
             pw[w4] = e4m3x4(pv[0] * cpv, pv[1] * cpv, pv[2] * cpv, pv[3] * cpv);
@@ -429,12 +452,14 @@ __global__ void __launch_bounds__(kNvThreads, 1)
       tc_fence_after();
       const float fin = (svmax / 448.0f) / l_row;
       const size_t orow = hrow + (size_t)qrow;
+      const bool store = !kShortTail || qrow < N;
 #pragma unroll 1
       for (int c = 0; c < 2; ++c) {
         uint32_t o[32];
         const int col = 64 * hf + 32 * c;
         tmem_ld32(tO + (uint32_t)col, o);
         tmem_wait_ld();
+        if (!store) continue;
         if (p.out_f32) {
           float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow * 128 + col);
 #pragma unroll

@@ -539,7 +539,6 @@ fqa_status fqa_attention_nvfp4(const uint8_t* q4, const uint8_t* k4, const uint8
                                fqa_out_dtype out_dtype, void* cuda_stream) {
   fqa_status st = check_attention_common(B, H, N, d, softmax_scale, out, out_dtype);
   if (st != FQA_OK) return st;
-  if (N % kBlockN != 0) return FQA_ERR_UNSUPPORTED;
   const void* ptrs[] = {q4, k4, sfq, sfk, sq1, sk1, v8, sv, sv_max};
   for (const void* p : ptrs)
     if (p == nullptr) return FQA_ERR_INVALID_ARG;
@@ -557,16 +556,19 @@ fqa_status fqa_attention_nvfp4(const uint8_t* q4, const uint8_t* k4, const uint8
   if (!make_tmap_fp4(&tq, q4, N, heads) || !make_tmap_fp4(&tk, k4, N, heads) ||
       !make_tmap(&tv, v8, true, N, heads))
     return FQA_ERR_CUDA;
-  if (cudaFuncSetAttribute(attn_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           NvTraits::kSmemBytes) != cudaSuccess)
+  // the short-tail instance only when N is not a multiple of 128
+  const bool tail = N % kBlockN != 0;
+  using NvKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const NvParams);
+  const NvKernel fn = tail ? attn_nvfp4_kernel<true> : attn_nvfp4_kernel<false>;
+  if (cudaFuncSetAttribute((const void*)fn, cudaFuncAttributeMaxDynamicSharedMemorySize, NvTraits::kSmemBytes) !=
+      cudaSuccess)
     return FQA_ERR_CUDA;
   NvParams prm{B, H, N, softmax_scale, sfq, sfk, sq1, sk1, sv, sv_max, out, out_dtype == FQA_OUT_F32, status};
-  const int items = heads * (N / kBlockM);
+  const int items = heads * ((N + kBlockM - 1) / kBlockM);
   const int sms = num_sms();
   if (sms <= 0) return FQA_ERR_CUDA;
   const int grid = items < sms ? items : sms;
-  attn_nvfp4_kernel<<<grid, kNvThreads, NvTraits::kSmemBytes, static_cast<cudaStream_t>(cuda_stream)>>>(
-      tq, tk, tv, prm);
+  fn<<<grid, kNvThreads, NvTraits::kSmemBytes, static_cast<cudaStream_t>(cuda_stream)>>>(tq, tk, tv, prm);
   return launch_status();
 }
 

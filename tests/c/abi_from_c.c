@@ -39,7 +39,7 @@ int main(void) {
         FQA_ERR_INVALID_ARG);
   CHECK(fqa_e4m3_encode(NULL, (uint8_t*)p, 4, NULL) == FQA_ERR_INVALID_ARG);
   uint8_t* u = (uint8_t*)p;
-  CHECK(fqa_attention_nvfp4(u, u, u, u, f, f, p, f, f, 1, 1, 200, 128, 0.088f, p, FQA_OUT_BF16, NULL) ==
+  CHECK(fqa_attention_nvfp4(u, u, u, u, f, f, p, f, f, 1, 1, 200, 64, 0.088f, p, FQA_OUT_BF16, NULL) ==
         FQA_ERR_UNSUPPORTED);
   CHECK(fqa_quantize_nvfp4_qk(p, p, f, 1, 1, 128, 128, NULL, u, u, u, f, f, NULL) == FQA_ERR_INVALID_ARG);
   CHECK(fqa_e2m1_encode(NULL, u, 4, NULL) == FQA_ERR_INVALID_ARG);

@@ -10,7 +10,7 @@ V projections; attention itself stays in FP8).
 - fqa_attention_nvfp4: every element within 1e-2 + amb of the oracle (amb:
   the oracle's bound on P codes the binary32 evaluation may round either
   way), mean relative error <= 2e-3 -- the FP8 path's bar; all rows on the
-  small cases, sampled rows at full size.
+  small cases, sampled rows at full size; any sequence length.
 """
 
 import numpy as np
@@ -181,18 +181,30 @@ def test_attention_nvfp4_degenerate_cases():
     assert torch.count_nonzero(out) == 0
 
 
-def test_attention_nvfp4_deterministic_and_rejects_ragged():
+def test_attention_nvfp4_deterministic():
     fqa = _fqa()
     g = U.host_inputs(1)
     qz, qn = _gpu_nvfp4(g)
     a = fqa.attention_nvfp4(qn, qz, U.SCALE)
     b = fqa.attention_nvfp4(qn, qz, U.SCALE)
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
-    shape = (1, 1, 200, 128)
-    bits = {t: _gen(shape, 40 + i) for i, t in enumerate("qkv")}
+
+
+@pytest.mark.parametrize("N", [1, 63, 100, 129, 200, 1000, 4429])
+def test_attention_nvfp4_ragged(N):
+    """Any sequence length: the short last Q tile and KV tile (keys past N
+    take no part; the second 64-key half of the last tile may be empty),
+    every row against the oracle on the small cases, sampled rows on 4429."""
+    fqa = _fqa()
+    shape = (1, 3, N, 128)
+    bits = {t: _gen(shape, 30 + i, 2.0) for i, t in enumerate("qkv")}
     qz, qn = _gpu_nvfp4(bits)
-    with pytest.raises(fqa.FqaError):
-        fqa.attention_nvfp4(qn, qz, U.SCALE)
+    out = fqa.attention_nvfp4(qn, qz, U.SCALE, fqa.FQA_OUT_F32).cpu().numpy()
+    assert fqa.fqa_debug_status()[0] == fqa.FQA_OK
+    rows = list(range(N)) if N <= 1000 else U.sample_rows(N)
+    ref, amb, _ = oracle.attention_nvfp4(_as_oracle(qz, qn), U.SCALE, rows=rows, with_ambiguity=True)
+    got = out[:, :, rows].reshape(ref.shape)
+    _compare(got, ref, amb)
 
 
 def test_nvfp4_tracks_fp8_on_workload():
