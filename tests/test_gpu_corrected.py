@@ -197,3 +197,31 @@ def test_patched_tiles_extreme_blocks(layout):
     m = U.metrics(got, ref)
     assert m["mean_rel"] <= 2e-3, m
     assert np.all(np.abs(got - ref) <= 1e-2 + amb), float((np.abs(got - ref) - amb).max())
+
+
+@pytest.mark.parametrize("rho", [0.0005, 0.005])
+def test_corrected_longest_sequence_sampled(rho):
+    """N = 65536 (the maximum), one head: 33 corrected keys (patched FP8 part)
+    and 328 (key-masked FP8 part, exact part in three chunks); the selection
+    reads the errors from global memory at this length.  Sampled rows."""
+    fqa = _fqa()
+    N = 65536
+    rng = np.random.default_rng(77)
+    g = {t: synth.round_to_bf16_bits(rng.standard_normal((1, 1, N, 128)) * s)
+         for t, s in zip("qkv", (2.0, 2.0, 1.0))}
+    q, k, v = (U.to_device(g[t]) for t in "qkv")
+    qz, k_err = fqa.quantize_keyerr(q, k, v)
+    out32 = fqa.attention_fp8_corrected(q, k, v, qz, k_err, U.SCALE, rho, fqa.FQA_OUT_F32).cpu().numpy()
+    assert fqa.fqa_debug_status()[0] == fqa.FQA_OK
+    oq = oracle.quantize(g["q"], g["k"], g["v"])
+    kc = oracle.n_corrected(N, rho)
+    assert kc == fqa.fqa_corrected_keys(N, rho)
+    err = oracle.key_error(g["k"], oq)
+    assert np.array_equal(err.view(np.uint32), k_err.cpu().numpy().view(np.uint32))
+    sel = oracle.select_keys(err, kc)
+    rows = [0, 1, 63, 64, 127, 128, N // 2, N - 129, N - 64, N - 1]
+    ref, amb = oracle.attention_fp8_corrected(g, oq, sel, U.SCALE, rows=rows, with_ambiguity=True)
+    got = out32[0, 0][rows].astype(np.float64)[None]
+    m = U.metrics(got, ref)
+    assert m["mean_rel"] <= 2e-3, m
+    assert np.all(np.abs(got - ref) <= 1e-2 + amb), float((np.abs(got - ref) - amb).max())

@@ -222,3 +222,16 @@ def test_nvfp4_tracks_fp8_on_workload():
     cos = float((got * ex[0]).sum() / np.sqrt((got * got).sum() * (ex[0] * ex[0]).sum()))
     print(f"\n[{w.name}] nvfp4 cos vs exact (head 0, sampled rows): {cos:.4f}")
     assert cos > 0.9
+
+
+def test_attention_nvfp4_longest_sequence_sampled():
+    """N = 65536 (the maximum), one head, sampled rows against all keys."""
+    fqa = _fqa()
+    N = 65536
+    bits = {t: _gen((1, 1, N, 128), 55 + i) for i, t in enumerate("qkv")}
+    qz, qn = _gpu_nvfp4(bits)
+    out = fqa.attention_nvfp4(qn, qz, U.SCALE, fqa.FQA_OUT_F32).cpu().numpy()
+    assert fqa.fqa_debug_status()[0] == fqa.FQA_OK
+    rows = [0, 1, 63, 64, 127, 128, N // 2, N - 129, N - 64, N - 1]
+    ref, amb, _ = oracle.attention_nvfp4(_as_oracle(qz, qn), U.SCALE, rows=rows, with_ambiguity=True)
+    _compare(out[0, 0][rows][None], ref, amb)
