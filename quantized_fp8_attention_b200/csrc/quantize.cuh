@@ -140,57 +140,121 @@ __device__ __forceinline__ float residual_sq8(const float* x, const uint32_t (&w
   return acc;
 }
 
-// Block absmax over the CTA (red: one float per warp, in buffer `slot`),
-// scale, and the codes of this thread's chunks (8 bytes per chunk, chunk c at
-// byte 8c; chunks at or beyond nvalid are not stored).  The CTA-wide sync of
-// the absmax also combines `ok` (this thread's wait for the unit): unless
-// every thread's is true nothing is stored and false is returned.  It is the
-// unit's one sync: the caller's slot may be refilled after it (x holds the
-// values) and the other `red` buffer is free for the next unit.  rsq
-// (optional): each chunk's residual squares (residual_sq8).
-__device__ __forceinline__ bool quantize_chunks(float (&x)[kVals], float* red, uint8_t* dst, int slot,
+// Lane-wise max(|a|, |b|) of two BF16 pairs: max.xorsign.abs leaves that
+// magnitude in each lane (the sign bit, an XOR of the inputs', is not used),
+// so a tree of them ends with the largest magnitude of each lane.
+__device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// BF16 pair (element 0 in the low half) -> its two exact binary32 values.
+__device__ __forceinline__ float2 bf16x2_to_f2(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+
+// The largest |x| over the CTA, from this thread's m >= 0 (red: one float
+// per warp, in buffer `slot`; non-negative binary32 values order like their
+// bit patterns, so the warp maximum is an integer reduction), and the block's
+// scale and inverse.  The CTA-wide sync also combines `ok` (this thread's
+// wait for the unit): unless every thread's is true, false is returned.  It
+// is the unit's one sync: the caller's slot may be refilled after it and the
+// other `red` buffer is free for the next unit.
+__device__ __forceinline__ bool block_scale(float m, float* red, int slot, bool ok, float& scale,
+                                            float& inv) {
+  const int t = threadIdx.x;
+  const uint32_t mw = __reduce_max_sync(0xffffffffu, __float_as_uint(m));
+  if ((t & 31) == 0) red[slot * kQuantWarps + (t >> 5)] = __uint_as_float(mw);
+  if (!__syncthreads_and(ok)) return false;
+  static_assert(kQuantWarps == 8, "two float4 loads per buffer");
+  const float4 r0 = *reinterpret_cast<const float4*>(red + slot * kQuantWarps);
+  const float4 r1 = *reinterpret_cast<const float4*>(red + slot * kQuantWarps + 4);
+  const float a = fmax3(fmax3(r0.x, r0.y, r0.z), fmax3(r0.w, r1.x, r1.y), fmaxf(r1.z, r1.w));
+  scale = a > 0.0f ? __fdiv_rn(a, 448.0f) : 0.0f;
+  inv = a > 0.0f ? __fdiv_rn(448.0f, a) : 0.0f;
+  if (scale == 0.0f) inv = 0.0f;               // amax / 448 underflowed: flush the block
+  return true;
+}
+
+// Codes of 8 values (one chunk) -> two words, value 0 in bits [0,8): x * inv,
+// or x / scale where inv overflowed (amax below about 1.3e-36, block-uniform:
+// the block's zeros then stay zeros instead of 0 * inf).
+__device__ __forceinline__ uint2 chunk_codes(const float (&x)[8], float scale, float inv) {
+  if (isinf(inv)) {
+    return make_uint2(e4m3x4(__fdiv_rn(x[0], scale), __fdiv_rn(x[1], scale), __fdiv_rn(x[2], scale),
+                             __fdiv_rn(x[3], scale)),
+                      e4m3x4(__fdiv_rn(x[4], scale), __fdiv_rn(x[5], scale), __fdiv_rn(x[6], scale),
+                             __fdiv_rn(x[7], scale)));
+  }
+  const float2 i2 = make_float2(inv, inv);
+  const float2 p0 = f2_mul(make_float2(x[0], x[1]), i2), p1 = f2_mul(make_float2(x[2], x[3]), i2);
+  const float2 p2 = f2_mul(make_float2(x[4], x[5]), i2), p3 = f2_mul(make_float2(x[6], x[7]), i2);
+  return make_uint2(e4m3x4(p0.x, p0.y, p1.x, p1.y), e4m3x4(p2.x, p2.y, p3.x, p3.y));
+}
+
+// Block absmax, scale and the codes of this thread's chunks of a staged BF16
+// unit (raw: the chunks as loaded; chunks at or beyond nvalid are zeros and
+// are not stored; chunk c's 8 codes go to byte 8c of dst).  The absmax is
+// taken on the BF16 pairs (BF16 -> binary32 is exact, so it is the binary32
+// absmax); the values are converted after the sync.
+__device__ __forceinline__ bool quantize_chunks_bf16(const uint4 (&raw)[kChunks], float* red, uint8_t* dst,
+                                                     int slot, int nvalid, uint64_t policy, bool ok,
+                                                     float& scale_out) {
+  const int t = threadIdx.x;
+  static_assert(kChunks == 4, "a 16-word tree");
+  uint32_t w[8];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    w[4 * i + 0] = bf16x2_absmax(raw[i].x, raw[i + 2].x);
+    w[4 * i + 1] = bf16x2_absmax(raw[i].y, raw[i + 2].y);
+    w[4 * i + 2] = bf16x2_absmax(raw[i].z, raw[i + 2].z);
+    w[4 * i + 3] = bf16x2_absmax(raw[i].w, raw[i + 2].w);
+  }
+  const uint32_t w4 = bf16x2_absmax(bf16x2_absmax(w[0], w[4]), bf16x2_absmax(w[1], w[5]));
+  const uint32_t w5 = bf16x2_absmax(bf16x2_absmax(w[2], w[6]), bf16x2_absmax(w[3], w[7]));
+  const float2 mf = bf16x2_to_f2(bf16x2_absmax(w4, w5));
+  float scale, inv;
+  if (!block_scale(fmaxf(fabsf(mf.x), fabsf(mf.y)), red, slot, ok, scale, inv)) return false;
+#pragma unroll
+  for (int i = 0; i < kChunks; ++i) {
+    float x[8];
+    const uint32_t ww[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = bf16x2_to_f2(ww[e]);
+      x[2 * e] = f.x;
+      x[2 * e + 1] = f.y;
+    }
+    const uint2 c = chunk_codes(x, scale, inv);
+    if (t + kQuantThreads * i < nvalid) st_global_v2_hint(dst + 8 * (t + kQuantThreads * i), c.x, c.y, policy);
+  }
+  scale_out = scale;
+  return true;
+}
+
+// The same for binary32 values x (this thread's chunks, chunk i in x[8i..8i+8);
+// values of chunks past nvalid must be zeros).  rsq (optional): each chunk's
+// residual squares (residual_sq8).
+__device__ __forceinline__ bool quantize_chunks(const float (&x)[kVals], float* red, uint8_t* dst, int slot,
                                                 int nvalid, uint64_t policy, bool ok, float& scale_out,
                                                 float* rsq = nullptr) {
   const int t = threadIdx.x;
-  float m = 0.0f;
+  static_assert(kVals == 32, "a 32-value tree");
+  float m[11];
 #pragma unroll
-  for (int i = 0; i < kVals; ++i) m = fmaxf(m, fabsf(x[i]));
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if ((t & 31) == 0) red[slot * kQuantWarps + (t >> 5)] = m;
-  if (!__syncthreads_and(ok)) return false;
-  float a = red[slot * kQuantWarps];
-#pragma unroll
-  for (int w = 1; w < kQuantWarps; ++w) a = fmaxf(a, red[slot * kQuantWarps + w]);
-  const float scale = a > 0.0f ? __fdiv_rn(a, 448.0f) : 0.0f;
-  float inv = a > 0.0f ? __fdiv_rn(448.0f, a) : 0.0f;
-  if (scale == 0.0f) inv = 0.0f;               // amax / 448 underflowed: flush the block
-  if (isinf(inv)) {
-    // 448 / amax overflowed (amax below about 1.3e-36): codes of x / scale,
-    // so the block's zeros stay zeros instead of 0 * inf.  Block-uniform.
-#pragma unroll
-    for (int i = 0; i < kChunks; ++i) {
-      uint32_t w[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        w[e] = e4m3x2(__fdiv_rn(x[8 * i + 2 * e], scale), __fdiv_rn(x[8 * i + 2 * e + 1], scale));
-      if (t + kQuantThreads * i < nvalid)
-        st_global_v2_hint(dst + 8 * (t + kQuantThreads * i), w[0] | (w[1] << 16), w[2] | (w[3] << 16), policy);
-      if (rsq) rsq[i] = residual_sq8(&x[8 * i], w, scale);
-    }
-    scale_out = scale;
-    return true;
-  }
+  for (int i = 0; i < 10; ++i) m[i] = fmax3(fabsf(x[3 * i]), fabsf(x[3 * i + 1]), fabsf(x[3 * i + 2]));
+  m[10] = fmaxf(fabsf(x[30]), fabsf(x[31]));
+  const float m0 = fmax3(fmax3(m[0], m[1], m[2]), fmax3(m[3], m[4], m[5]), fmax3(m[6], m[7], m[8]));
+  float scale, inv;
+  if (!block_scale(fmax3(m0, m[9], m[10]), red, slot, ok, scale, inv)) return false;
 #pragma unroll
   for (int i = 0; i < kChunks; ++i) {
-    uint32_t lo = e4m3x2(__fmul_rn(x[8 * i], inv), __fmul_rn(x[8 * i + 1], inv));
-    uint32_t hi = e4m3x2(__fmul_rn(x[8 * i + 2], inv), __fmul_rn(x[8 * i + 3], inv));
-    uint32_t lo2 = e4m3x2(__fmul_rn(x[8 * i + 4], inv), __fmul_rn(x[8 * i + 5], inv));
-    uint32_t hi2 = e4m3x2(__fmul_rn(x[8 * i + 6], inv), __fmul_rn(x[8 * i + 7], inv));
-    if (t + kQuantThreads * i < nvalid)
-      st_global_v2_hint(dst + 8 * (t + kQuantThreads * i), lo | (hi << 16), lo2 | (hi2 << 16), policy);
+    const float(&xc)[8] = *reinterpret_cast<const float(*)[8]>(&x[8 * i]);
+    const uint2 c = chunk_codes(xc, scale, inv);
+    if (t + kQuantThreads * i < nvalid) st_global_v2_hint(dst + 8 * (t + kQuantThreads * i), c.x, c.y, policy);
     if (rsq) {
-      const uint32_t w[4] = {lo, hi, lo2, hi2};
+      const uint32_t w[4] = {c.x & 0xFFFFu, c.x >> 16, c.y & 0xFFFFu, c.y >> 16};
       rsq[i] = residual_sq8(&x[8 * i], w, scale);
     }
   }
@@ -210,7 +274,7 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantMinCtas) quantize_fused_k
   uint8_t* side = ring + kRingBytes;               // kMaxSlots x kSideBytes
   __shared__ uint64_t full[kMaxSlots];
   __shared__ int slot_unit[kMaxSlots];
-  __shared__ float red[2 * kQuantWarps];
+  __shared__ __align__(16) float red[2 * kQuantWarps];
   __shared__ int failed, abort_flag;
   const int t = threadIdx.x;
   const int nblk = (N + kQBlock - 1) / kQBlock;
@@ -317,10 +381,14 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantMinCtas) quantize_fused_k
         },
         [&](int u, const uint8_t* blk, bool ok, int par) -> bool {
           const int nvalid = unit_rows(u) * (kHeadDim * 2 / 16);
-          float x[kVals];
-          chunks_to_f32(blk, nvalid, x);
+          uint4 raw[kChunks];
+#pragma unroll
+          for (int i = 0; i < kChunks; ++i) {
+            const int c = t + kQuantThreads * i;
+            raw[i] = c < nvalid ? *reinterpret_cast<const uint4*>(blk + 16 * c) : make_uint4(0, 0, 0, 0);
+          }
           float sc;
-          if (!quantize_chunks(x, red, codes + unit_off(u), par, nvalid, pol_first, ok, sc)) return false;
+          if (!quantize_chunks_bf16(raw, red, codes + unit_off(u), par, nvalid, pol_first, ok, sc)) return false;
           if (t == 0) scales[u] = sc;
           return true;
         });
@@ -420,9 +488,10 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantMinCtas) quantize_fused_k
         // every chunk of this thread starts at channel 8t mod 128
         const float* mu = reinterpret_cast<const float*>(side + (blk - ring) / kBlockBytes * kSideBytes) +
                           ((8 * t) & (kHeadDim - 1));
-        float mr[8];
+        // x - mu as x + (-mu): the same IEEE result, two channels per add
+        float2 nmu[4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) mr[e] = mu[e];
+        for (int e = 0; e < 4; ++e) nmu[e] = make_float2(-mu[2 * e], -mu[2 * e + 1]);
         const int nvalid = unit_rows(u) * (kHeadDim * 2 / 16);
         float x[kVals];
         chunks_to_f32(blk, nvalid, x);
@@ -431,7 +500,11 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantMinCtas) quantize_fused_k
           // chunks past a short block's tokens stay 0: they must not enter amax
           if (t + kQuantThreads * i4 < nvalid) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) x[8 * i4 + e] = __fsub_rn(x[8 * i4 + e], mr[e]);
+            for (int e = 0; e < 4; ++e) {
+              const float2 d = f2_add(make_float2(x[8 * i4 + 2 * e], x[8 * i4 + 2 * e + 1]), nmu[e]);
+              x[8 * i4 + 2 * e] = d.x;
+              x[8 * i4 + 2 * e + 1] = d.y;
+            }
           }
         }
         float s_k;
