@@ -481,8 +481,9 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantMinCtas) quantize_fused_k
         const uint32_t bytes = (uint32_t)unit_rows(u) * kHeadDim * 2;
         mbar_arrive_expect_tx(bar, bytes + kSideBytes);
         bulk_load(dst, k + unit_in(u), bytes, bar, pol_first);
+        // (the row is read again by every unit of its head: it stays in L2)
         bulk_load(side + (dst - ring) / kBlockBytes * kSideBytes, k_mean + (size_t)(u / nblk) * kHeadDim,
-                  kSideBytes, bar, pol_first);
+                  kSideBytes, bar, pol_last);
       },
       [&](int u, const uint8_t* blk, bool ok, int par) -> bool {
         // every chunk of this thread starts at channel 8t mod 128
